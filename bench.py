@@ -1,0 +1,458 @@
+"""Benchmark: block top-k sparse decode over a paged KV cache on B200 (req-heads/s).
+
+One step = one decode layer of the Qwen3-0.6B-like workload (B=32, Hq=16, Hkv=8, D=128,
+page 16, contexts U[4096, 16384], 40,000-page shuffled pool, top-30 + 1 + 1 pages):
+  vt_build_centroids  on the pages that fill at this step (requests whose length is a
+                      multiple of 16),
+  vt_plan_requests    request order, longest first,
+  vt_sparse_decode_fused  group mean -> centroid scores -> exact top-k + reserved pages ->
+                      attention over the selected pages, one launch.
+Inputs are resident in HBM; steps rotate over ``--replicas`` copies of the inputs (pools,
+centroids, q, page tables) whose combined footprint is far above the 126 MB L2, so no step
+finds its data in L2.  Rank 0 prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+``--impl reference`` times the fp64 CPU oracle on this host's cores on the same workload
+(each step a bounded sample of requests) -- the only other place this script runs it is the
+``cpu_baseline`` leg of the default arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_block_sparse_vt_b200.workloads import PAGE_SIZE, config, make_workload  # noqa: E402
+
+CFG = 2
+METRIC = "sparse-decode req-heads/s"
+UNIT = "req-heads/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fused_kernel_traffic.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ------------------------------------------------------------------------------------------
+# algorithmic bytes (what the method must move; not the dense KV it avoids)
+# ------------------------------------------------------------------------------------------
+def algorithmic_bytes(c, seq_lens: torch.Tensor) -> dict:
+    """Per step, from the generated lengths:
+    fused   = sum_b [2 Hq D (q) + 2 Hq Dv (out) + 4 Hq (lse) + 4 n_b (page-table row)]
+            + sum_{b,h} [4 D |C_b| (candidate centroids, sparse requests only)
+                         + 2 (D + Dv) * tokens of the selected pages]
+    build   = per filled page: 16 Hkv D * 2 (K read) + Hkv D * 4 (centroid write) + 4 (id)
+    With eos >= 1 the (possibly partial) last page is always selected, so the selected tokens
+    of a unit are 16 (min(n, kmax) - 1) + valid tokens of the last page.
+    """
+    assert c.eos >= 1
+    L = seq_lens.long()
+    n = (L + PAGE_SIZE - 1) // PAGE_SIZE
+    last_valid = L - PAGE_SIZE * (n - 1)
+    sparse = n > c.kmax
+    cand = torch.where(sparse, n - c.bos - c.eos, torch.zeros_like(n))
+    sel_pages = torch.minimum(n, torch.full_like(n, c.kmax))
+    tokens = PAGE_SIZE * (sel_pages - 1) + last_valid
+    per_req = 2 * c.Hq * c.D + 2 * c.Hq * c.Dv + 4 * c.Hq + 4 * n
+    per_unit = 4 * c.D * cand + 2 * (c.D + c.Dv) * tokens
+    fused = int(per_req.sum()) + c.Hkv * int(per_unit.sum())
+    n_fill = int((L % PAGE_SIZE == 0).sum())
+    build = n_fill * (PAGE_SIZE * c.Hkv * c.D * 2 + c.Hkv * c.D * 4 + 4)
+    return dict(fused=fused, build=build, total=fused + build,
+                centroid_bytes=c.Hkv * int((4 * c.D * cand).sum()),
+                kv_bytes=c.Hkv * int((2 * (c.D + c.Dv) * tokens).sum()))
+
+
+def read_peak_hbm():
+    try:
+        with open(PEAKS_FILE) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("decode_fma.cu", "common.cuh", "decode_params.cuh"):
+        with open(os.path.join(ROOT, "paged_block_sparse_vt_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the fused kernel from an ncu capture, if taken on this source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+        if rec.get("source_hash") == kernel_source_hash():
+            return rec.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; the data path has no collective)
+# ------------------------------------------------------------------------------------------
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif n_gpus > 1:
+        raise SystemExit("--gpus N > 1 needs torchrun (one process per GPU)")
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------------
+# the reference arm: the CPU oracle
+# ------------------------------------------------------------------------------------------
+def oracle_prepare(w):
+    import oracle
+    oracle.build()
+    c = w["config"]
+    cent = torch.full((w["P"], c.Hkv, c.D), float("nan"))
+    oracle.build_centroids(w["k_pool"], w["prebuilt_pages"], cent)
+    return cent
+
+
+def oracle_step(w, cent, reqs):
+    """One oracle decode step over the requests in ``reqs``: build the centroids of the pages
+    that fill at this step, then select + attend."""
+    import oracle
+    c = w["config"]
+    idx = torch.tensor(reqs, dtype=torch.long)
+    L = w["seq_lens"][idx]
+    n = (L + PAGE_SIZE - 1) // PAGE_SIZE
+    fill = [int(w["page_table"][b, int(n[i]) - 1]) for i, b in enumerate(reqs)
+            if int(L[i]) % PAGE_SIZE == 0]
+    if fill:
+        oracle.build_centroids(w["k_pool"], torch.tensor(fill, dtype=torch.int32), cent)
+    oracle.decode_step(w["q"][idx].contiguous(), w["k_pool"], w["v_pool"],
+                       w["page_table"][idx].contiguous(), L.contiguous(), cent, c.topk, c.bos,
+                       c.eos, c.sm_scale)
+
+
+def oracle_sample_size(w, cent, target_s: float) -> list:
+    """Requests per oracle step so that one step takes about target_s seconds (>= 1)."""
+    c = w["config"]
+    t0 = time.perf_counter()
+    oracle_step(w, cent, [0])
+    dt = max(1e-4, time.perf_counter() - t0)
+    k = max(1, min(c.B, int(target_s / dt)))
+    return list(range(k))
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return  # rank 0 alone runs the CPU reference
+    import oracle
+    c = config(CFG)
+    w = make_workload(c)
+    cent = oracle_prepare(w)
+    cores = oracle.get_threads()
+    reqs = oracle_sample_size(w, cent, target_s=max(0.5, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_step(w, cent, reqs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(w, cent, reqs)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = len(reqs) * c.Hq / dt
+    sample = (f"{len(reqs)} of {c.B} requests ({len(reqs) * c.Hq} req-heads) per step, fp64 C "
+              f"oracle, OpenMP over (request, KV head)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(c, w, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(c, w, args) -> dict:
+    return {
+        "workload": f"qwen3-0.6b-like sparse decode layer (B={c.B}, Hq={c.Hq}, Hkv={c.Hkv}, "
+                    f"D={c.D}, page 16, context U[{c.len_lo},{c.len_hi}], top-{c.topk}+{c.bos}+{c.eos})",
+        "B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "head_dim": c.D, "page_size": PAGE_SIZE,
+        "topk": c.topk, "bos": c.bos, "eos": c.eos, "pool_pages": w["P"],
+        "mean_pages_per_request": float(((w["seq_lens"].double() + 15) // 16).mean()),
+        "parallelism": f"dp{args.gpus} (independent batches per GPU)",
+        "l2": f"inputs rotate over {args.replicas} resident copies (>126 MB L2 between reuses)",
+    }
+
+
+# ------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    import paged_block_sparse_vt_b200 as vt
+    vt.load_library()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    c = config(CFG)
+    w = make_workload(c, seed=1000 + CFG + 7919 * rank)
+    nbytes = algorithmic_bytes(c, w["seq_lens"])
+    stream = torch.cuda.current_stream(dev)
+
+    # resident replicas of every per-step input; centroids of the full pages prebuilt
+    reps = []
+    for r in range(args.replicas):
+        d = {k: w[k].to(dev) for k in ("q", "k_pool", "v_pool", "page_table", "seq_lens",
+                                        "prebuilt_pages", "fill_pages")}
+        d["cent"] = torch.zeros((w["P"], c.Hkv, c.D), dtype=torch.float32, device=dev)
+        vt.vt_build_centroids(d["k_pool"], d["prebuilt_pages"], d["cent"])
+        d["out"] = torch.empty((c.B, c.Hq, c.Dv), dtype=torch.bfloat16, device=dev)
+        d["lse"] = torch.empty((c.B, c.Hq), dtype=torch.float32, device=dev)
+        d["order"] = torch.empty((c.B,), dtype=torch.int32, device=dev)
+        d["status"] = torch.zeros((1,), dtype=torch.int32, device=dev)
+        reps.append(d)
+    torch.cuda.synchronize(dev)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+
+    def step(d, i=None):
+        vt.vt_build_centroids(d["k_pool"], d["fill_pages"], d["cent"], status=d["status"])
+        if not args.no_plan:
+            vt.vt_plan_requests(d["seq_lens"], d["order"])
+        if i is not None:
+            ev[i][0].record(stream)
+        vt.vt_sparse_decode_fused(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                  d["seq_lens"], d["cent"], c.topk, c.bos, c.eos, c.sm_scale,
+                                  out=d["out"], lse=d["lse"],
+                                  order=None if args.no_plan else d["order"], status=d["status"])
+        if i is not None:
+            ev[i][1].record(stream)
+
+    launches_per_step = 2 + (0 if args.no_plan else 1)
+    for i in range(args.warmup):
+        step(reps[i % args.replicas])
+    torch.cuda.synchronize(dev)
+    barrier(world)
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(reps[i % args.replicas], i)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    elapsed = t_start.elapsed_time(t_end) / 1e3
+    fused_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    elapsed = max_over_ranks(elapsed, world, dev)
+
+    # end to end through the public API: pinned host inputs in, results back, every step
+    host = {k: w[k].pin_memory() for k in ("q", "page_table", "seq_lens", "fill_pages")}
+    out_h = torch.empty((c.B, c.Hq, c.Dv), dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.empty((c.B, c.Hq), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+
+    def e2e_step(d):
+        for k in host:
+            d[k].copy_(host[k], non_blocking=True)
+        step(d)
+        out_h.copy_(d["out"], non_blocking=True)
+        lse_h.copy_(d["lse"], non_blocking=True)
+        stream.synchronize()
+
+    for i in range(args.warmup):
+        e2e_step(reps[i % args.replicas])
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        e2e_step(reps[i % args.replicas])
+    e2e_s = max_over_ranks((time.perf_counter() - t0) / args.steps, world, dev)
+    clk = clocks.stop() if clocks else None
+
+    status = max(int(d["status"].item()) for d in reps)
+    if status:
+        raise SystemExit(f"device status {status}: an input was rejected by the kernels")
+
+    if rank != 0:
+        return
+    ms = elapsed / args.steps * 1e3
+    units = c.B * c.Hq
+    value = world * units * args.steps / elapsed
+    peak, peak_kind = read_peak_hbm()
+    achieved = nbytes["fused"] / (fused_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(c, w, args),
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": recorded_traffic(),
+            "kernel": "fma_decode_kernel (vt_sparse_decode_fused)",
+            "algorithmic_bytes_per_launch": nbytes["fused"], "kernel_ms": fused_ms,
+            "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
+            else "fallback 6650 GB/s",
+        },
+        "e2e": {"value": world * units / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "step_bytes": nbytes,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w) -> dict:
+    """The oracle, as it stands, on a bounded sample of the same workload (~15 s of CPU)."""
+    import oracle
+    c = w["config"]
+    cent = oracle_prepare(w)
+    reqs = oracle_sample_size(w, cent, target_s=5.0)
+    oracle_step(w, cent, reqs)  # warm
+    t0 = time.perf_counter()
+    reps = 0
+    while reps < 3 or time.perf_counter() - t0 < 10.0:
+        oracle_step(w, cent, reqs)
+        reps += 1
+        if time.perf_counter() - t0 > 30.0:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": len(reqs) * c.Hq / dt, "unit": UNIT, "cores": oracle.get_threads(),
+            "kind": "oracle",
+            "sample": f"{reps} oracle steps over requests 0..{len(reqs) - 1} of the same batch "
+                      f"({len(reqs) * c.Hq} req-heads each; build of filled pages + select + "
+                      f"attend), fp64"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--replicas", type=int, default=3)
+    ap.add_argument("--no-plan", action="store_true", help="skip the planner launch")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

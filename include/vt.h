@@ -1,0 +1,184 @@
+/*
+ * vt.h -- C ABI of libvt: block top-k sparse decode attention over a paged KV
+ * cache on NVIDIA B200 (sm_100a).
+ *
+ * The method (sources: "Vortex: A Flexible and Efficient Sparse Attention
+ * Framework", the vortex_torch README, sections "Quick Example: Custom Sparse
+ * Attention" and "Using Your Sparse Attention with SGLang"; and "Vortex:
+ * Efficient and Programmable Sparse Attention Serving for AI Agents", section
+ * "A dual-stage programmable abstraction"):
+ *   cache side  -- when a page of 16 tokens is finished, its centroid (the
+ *                  mean of its keys, one head_dim vector per KV head) is stored
+ *                  in a per-page cache;
+ *   query side  -- per request and KV head, the grouped query heads are
+ *                  averaged, the mean is scored against the centroid of every
+ *                  middle page, the top-k pages plus the reserved first `bos`
+ *                  and last `eos` pages are kept, and exact softmax attention
+ *                  runs over the tokens of those pages only.
+ *
+ * Conventions shared by every entry point
+ *   - Every data pointer is DEVICE memory owned by the caller.  The library
+ *     never allocates, frees or synchronises; each call enqueues its kernels
+ *     on `stream` (a cudaStream_t passed as void*; NULL = legacy default
+ *     stream) and returns.  No workspace is needed.
+ *   - bf16 means IEEE bfloat16 (upper half of a binary32), fp32 is binary32.
+ *   - Host-side argument checks fail fast with VT_ERR_INVALID_ARG or
+ *     VT_ERR_UNSUPPORTED before anything is launched; a failed launch returns
+ *     VT_ERR_CUDA.  vt_last_error_detail() gives a one-line reason (per host
+ *     thread).
+ *   - Checks that need device data (a page id outside [0, num_pages), a
+ *     seq_len < 1 or longer than the page table, a bad sel entry) are done by
+ *     the kernels: the affected unit is skipped (its outputs are zeroed) and
+ *     the matching VT_DEV_* bit is OR-ed into `*status` when a status word is
+ *     given.  Kernels never trap.
+ *   - Page size is 16 tokens.  Supported head shapes: (head_dim, head_dim_v) =
+ *     (64, 64) or (128, 128) with 1 <= Hq/Hkv <= 8, and the MLA latent form
+ *     (576, 512) with Hkv == 1, Hq in {16, 32} and v_pool == k_pool (V is the
+ *     first 512 dims of the K row, read from the same copy).
+ */
+#ifndef VT_H_
+#define VT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VT_ABI_VERSION 1
+#define VT_PAGE_SIZE 16
+#define VT_MAX_PAGES_PER_REQUEST 32768 /* page-table row length the kernels accept */
+
+typedef enum {
+  VT_OK = 0,
+  VT_ERR_INVALID_ARG = 1, /* null pointer, negative count, inconsistent sizes */
+  VT_ERR_UNSUPPORTED = 2, /* shape, stride or alignment with no kernel in this build */
+  VT_ERR_CUDA = 3         /* a CUDA runtime call or a kernel launch failed */
+} vt_status;
+
+/* Bits OR-ed into the optional device status word by the kernels. */
+#define VT_DEV_BAD_PAGE 1 /* a page id outside [0, num_pages); that unit/page was skipped */
+#define VT_DEV_BAD_LEN 2  /* seq_len < 1, or ceil(seq_len/16) > pt_stride; unit skipped */
+#define VT_DEV_BAD_SEL 4  /* n_sel or a sel entry out of range (vt_sparse_decode); unit skipped */
+
+/*
+ * Paged K/V layout ("vTensor" metadata, reduced to one descriptor).
+ * K element (page p, token t, kv head h, dim d) is
+ *   ((const bf16*)k_pool)[p*sk_p + t*sk_t + h*sk_h + d], d < head_dim;
+ * V element likewise with v_pool / sv_*, d < head_dim_v.  Strides are in
+ * elements; the innermost stride is 1.  Both pools must be 16-byte aligned
+ * and every stride a multiple of 8 elements (16 bytes).  For the MLA latent
+ * form, V is the first 512 dims of the K row: pass v_pool == k_pool and the
+ * same strides.
+ */
+typedef struct {
+  const void* k_pool;
+  const void* v_pool;
+  int64_t num_pages;    /* P: physical pages in the pool */
+  int32_t page_size;    /* must be VT_PAGE_SIZE */
+  int32_t num_kv_heads; /* Hkv */
+  int32_t head_dim;     /* D: query/key dimension */
+  int32_t head_dim_v;   /* Dv: value dimension */
+  int64_t sk_p, sk_t, sk_h;
+  int64_t sv_p, sv_t, sv_h;
+} vt_paged_kv;
+
+/*
+ * Per-step decode arguments.
+ *   q           bf16 [B, Hq, D], contiguous; query head hq belongs to KV head hq / (Hq/Hkv)
+ *   page_table  int32 [B, pt_stride]; entry (b, i) is the physical page of logical page i
+ *   seq_lens    int32 [B]; tokens of request b INCLUDING the one being decoded (its K/V is
+ *               already in the pool); logical pages n_b = ceil(seq_lens[b] / 16), the last
+ *               of which holds seq_lens[b] - 16 (n_b - 1) valid tokens
+ *   centroids   fp32 [P, Hkv, D], contiguous (vt_build_centroids output); read only for
+ *               the candidate pages [bos, n_b - eos) of requests with n_b > topk+bos+eos
+ *   topk, bos, eos  >= 0; kmax = topk + bos + eos.  A request with n_b <= kmax attends to
+ *               every page; otherwise to pages {0..bos-1} U {n_b-eos..n_b-1} U the topk
+ *               candidates with the highest score qm . centroid (ties -> lower index)
+ *   sm_scale    softmax scale applied to q . k (e.g. 1/sqrt(D))
+ *   order       optional int32 [B] permutation: the order in which requests are scheduled
+ *               (vt_plan_requests output); NULL = 0..B-1.  Results do not depend on it.
+ *   status      optional device int32 word receiving VT_DEV_* bits; NULL = not reported
+ */
+typedef struct {
+  int32_t batch;       /* B */
+  int32_t num_q_heads; /* Hq, a multiple of Hkv */
+  const void* q;
+  const int32_t* page_table;
+  int64_t pt_stride;
+  const int32_t* seq_lens;
+  const float* centroids;
+  int32_t topk, bos, eos;
+  float sm_scale;
+  const int32_t* order;
+  int32_t* status;
+} vt_decode_args;
+
+/*
+ * Cache side (README "Quick Example", forward_cache with CMean(dim=1), run
+ * when a page is finished; create_cache declares one (1, head_dim) centroid
+ * per page):  for each listed physical page p and KV head h,
+ *   centroids[p, h, :] = (1/16) * sum_{t<16} K[p, t, h, :]
+ * accumulated in fp64 and rounded once to fp32.  pages: int32 [n_pages]
+ * physical ids (the finished pages, "loc"); rows of other pages are not
+ * touched.  A listed id outside [0, num_pages) is skipped (VT_DEV_BAD_PAGE).
+ */
+vt_status vt_build_centroids(const vt_paged_kv* kv, const int32_t* pages, int32_t n_pages,
+                             float* centroids, int32_t* status, void* stream);
+
+/*
+ * Indexer (README "Quick Example", forward_indexer: q.mean -> GeMV against the
+ * centroids -> topK; reserved pages from vortex_page_reserved_bos/eos):
+ * writes, per request b and KV head h, the selected logical page indices in
+ * ascending order to sel[(b*Hkv + h)*kmax + j], j < n_sel[b*Hkv + h], and -1
+ * in the remaining slots.  sel: int32 [B, Hkv, kmax]; n_sel: int32 [B, Hkv].
+ * Scores are fp32 dot products of the fp32 group mean with the centroids.
+ */
+vt_status vt_select_pages(const vt_paged_kv* kv, const vt_decode_args* a, int32_t* sel,
+                          int32_t* n_sel, void* stream);
+
+/*
+ * Sparse attention over a given selection ("performs the actual attention" on
+ * the selected blocks through the paged layout): for each query head hq of
+ * request b, exact softmax(sm_scale * q K^T) V over the valid tokens of the
+ * logical pages sel[b, hq/G, 0:n_sel[b, hq/G]] (any order, no duplicates).
+ * out: bf16 [B, Hq, Dv]; lse: fp32 [B, Hq] natural-log sum of exp of the
+ * scaled scores, or NULL.  Accumulation is fp32.  a->centroids, topk/bos/eos
+ * are not used except kmax = topk+bos+eos, the row length of sel.
+ */
+vt_status vt_sparse_decode(const vt_paged_kv* kv, const vt_decode_args* a, const int32_t* sel,
+                           const int32_t* n_sel, void* out, float* lse, void* stream);
+
+/*
+ * The whole query side in one launch (selection + attention, "kernel fusion
+ * ... to minimize memory traffic", rndamp.com article, same section).  Same
+ * results as vt_select_pages followed by vt_sparse_decode.  sel / n_sel
+ * receive the selection when not NULL (both or neither).
+ */
+vt_status vt_sparse_decode_fused(const vt_paged_kv* kv, const vt_decode_args* a, void* out,
+                                 float* lse, int32_t* sel, int32_t* n_sel, void* stream);
+
+/*
+ * Workload planner ("a workload planner for balanced GPU scheduling", same
+ * article and section): writes to order[0..B) the request indices sorted by
+ * page count, longest first (equal counts keep index order), so that long
+ * scans start first.  The order can be computed once per decode step and
+ * reused by every layer.  seq_lens, order: device int32 [B]; B <= 65536.
+ */
+vt_status vt_plan_requests(const int32_t* seq_lens, int32_t batch, int32_t* order, void* stream);
+
+/* Static name of a status code. */
+const char* vt_status_string(vt_status s);
+
+/* One-line reason for the last non-OK status returned on this host thread ("" if none). */
+const char* vt_last_error_detail(void);
+
+/* VT_ABI_VERSION of the loaded library. */
+int32_t vt_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VT_H_ */

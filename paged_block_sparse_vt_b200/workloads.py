@@ -67,6 +67,7 @@ class Config:
     page_offsets: float     # std of the per-(page, head) offset added to K and V (0: none)
     mla: bool = False       # V is the first Dv dims of the K row (one shared pool)
     filled: int = 0         # requests whose last page fills at this step (cfg 5 recipe)
+    explicit: tuple = ()    # lengths="explicit": the seq_lens themselves (edge-case batches)
 
     @property
     def G(self) -> int:
@@ -104,6 +105,9 @@ def config(cfg: int, **overrides) -> Config:
 def _seq_lens(c: Config, gen: torch.Generator) -> torch.Tensor:
     if c.lengths == "fixed":
         L = torch.full((c.B,), c.len_lo, dtype=torch.int64)
+    elif c.lengths == "explicit":
+        assert len(c.explicit) == c.B
+        L = torch.tensor(c.explicit, dtype=torch.int64)
     elif c.lengths == "uniform":
         L = torch.randint(c.len_lo, c.len_hi + 1, (c.B,), generator=gen, dtype=torch.int64)
     elif c.lengths == "loguniform":
