@@ -191,6 +191,12 @@ def barrier(world):
         dist.barrier()
 
 
+def aggregate_value(world: int, units_per_rank: int, steps: int, elapsed_s: float) -> float:
+    """Whole-job throughput: every rank processed its own batch of units each step (weak
+    scaling); the time is the slowest rank's."""
+    return world * units_per_rank * steps / elapsed_s
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     if world == 1:
         return x
@@ -381,7 +387,7 @@ def run_ours(args, world, rank, local):
         return
     ms = elapsed / args.steps * 1e3
     units = c.B * c.Hq
-    value = world * units * args.steps / elapsed
+    value = aggregate_value(world, units, args.steps, elapsed)
     peak, peak_kind = read_peak_hbm()
     achieved = nbytes["fused"] / (fused_ms / 1e3) / 1e9
     line = {
