@@ -10,9 +10,9 @@
 namespace vt {
 cudaError_t launch_build_centroids(const vt_paged_kv& kv, const int32_t* pages, int n_pages,
                                    float* centroids, int32_t* status, cudaStream_t stream);
-cudaError_t launch_fma_decode(const DecodeParams& p, int mode, int D, int G, int C,
+cudaError_t launch_gqa_decode(const DecodeParams& p, int mode, int D, int G, int C,
                               cudaStream_t s);
-int fma_smem_bytes(int D, int G, int cand_cap, int key_cap, int kmax);
+int gqa_smem_bytes(int D, int G, int cand_cap, int key_cap, int kmax);
 cudaError_t launch_mla_decode(const DecodeParams& p, int mode, int G, int C, cudaStream_t s);
 int mla_smem_bytes(int G, int cand_cap, int key_cap, int kmax, int pages_per_cta);
 int mla_max_pages_per_cta();
@@ -44,7 +44,7 @@ vt_status cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-enum Path { kPathFma = 1, kPathMla = 2 };
+enum Path { kPathGqa = 1, kPathMla = 2 };
 
 struct Shape {
   Path path;
@@ -85,7 +85,7 @@ vt_status classify(const vt_paged_kv* kv, int Hq, Shape* sh) {
   const int D = kv->head_dim, Dv = kv->head_dim_v;
   if ((D == 64 || D == 128) && Dv == D) {
     if (G > 8) return fail(VT_ERR_UNSUPPORTED, "GQA group %d > 8 with head_dim %d", G, D);
-    *sh = Shape{kPathFma, D, Dv, G};
+    *sh = Shape{kPathGqa, D, Dv, G};
     return ok();
   }
   if (D == 576 && Dv == 512) {
@@ -123,10 +123,13 @@ int pick_cluster(const Shape& sh, int64_t units, int kmax) {
     while (C < 16 && (kmax + C - 1) / C > mla_max_pages_per_cta()) C *= 2;
     return C;
   }
-  const int64_t slots = (int64_t)sm_count() * 4;  // CTAs of 128 threads resident at once
-  if (units * 8 <= slots * 4) return 8;
-  if (units * 4 <= slots * 4) return 4;
-  return 4;
+  // One deep CTA per unit as soon as the units alone cover every SM (fewer, longer
+  // pipelines beat more, shorter ones); otherwise split units so that every SM has work.
+  const int64_t sms = sm_count();
+  if (units >= sms) return 1;
+  if (units * 2 >= sms) return 2;
+  if (units * 4 >= sms) return 4;
+  return 8;
 }
 
 vt_status fill_params(const vt_paged_kv* kv, const vt_decode_args* a, bool need_centroids,
@@ -204,10 +207,10 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
   p.cand_cap = (max_cand + C - 1) / C;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (sh.path == kPathFma) {
-    const int bytes = fma_smem_bytes(sh.D, sh.G, p.cand_cap, p.key_cap, p.kmax);
+  if (sh.path == kPathGqa) {
+    const int bytes = gqa_smem_bytes(sh.D, sh.G, p.cand_cap, p.key_cap, p.kmax);
     if (bytes > 227 * 1024) return fail(VT_ERR_UNSUPPORTED, "shared memory need %d B too large", bytes);
-    e = launch_fma_decode(p, mode, sh.D, sh.G, C, st);
+    e = launch_gqa_decode(p, mode, sh.D, sh.G, C, st);
   } else {
     const int ppc = (p.kmax + C - 1) / C;
     if (ppc > mla_max_pages_per_cta())

@@ -62,129 +62,6 @@ __device__ __forceinline__ void flag(int32_t* status, int bits) {
   if (status) atomicOr(status, bits);
 }
 
-// ---- block-wide exclusive scan (NT threads, scratch >= NT/32 ints) ---------------------
-template <int NT>
-__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch) {
-  constexpr int NW = NT / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(kFull, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) scratch[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < NW ? scratch[lane] : 0;
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(kFull, wi, o);
-      if (lane >= o) wi += y;
-    }
-    if (lane < NW) scratch[lane] = wi - w;
-  }
-  __syncthreads();
-  int res = scratch[warp] + x - v;
-  __syncthreads();
-  return res;
-}
-
-// ---- exact top-k by radix select over 32-bit keys ---------------------------------------
-// Finds the k-th largest key (k >= 1, k <= m) of keys[0..m) with 8-bit digits, most
-// significant first.  On return: every key whose masked value is > prefix is in the top-k;
-// keys whose masked value == prefix are all in it when take_all, else (mask is full) the
-// `need` lowest-index ones are.  hist: 256 ints; info: 4 ints (shared).
-template <int NT>
-__device__ void radix_select(const uint32_t* keys, int m, int k, int* hist, int* info,
-                             uint32_t& prefix, uint32_t& mask, int& need, bool& take_all) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  prefix = 0;
-  mask = 0;
-  need = k;
-  take_all = false;
-#pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += NT) hist[i] = 0;
-    __syncthreads();
-    for (int j = tid; j < m; j += NT) {
-      const uint32_t key = keys[j];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      int cnt[8], tot = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        cnt[i] = hist[8 * lane + i];
-        tot += cnt[i];
-      }
-      int incl = tot;  // sum over lanes >= lane (bins at or above this lane's)
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_down_sync(kFull, incl, o);
-        if (lane + o < 32) incl += y;
-      }
-      const int above_lane = incl - tot;
-      if (above_lane < need && need <= incl) {
-        int acc = above_lane;
-#pragma unroll
-        for (int i = 7; i >= 0; --i) {
-          if (acc + cnt[i] >= need) {
-            info[0] = 8 * lane + i;
-            info[1] = acc;
-            info[2] = cnt[i];
-            break;
-          }
-          acc += cnt[i];
-        }
-      }
-    }
-    __syncthreads();
-    const int d = info[0], above = info[1], cnt_d = info[2];
-    prefix |= (uint32_t)d << shift;
-    mask |= 0xffu << shift;
-    need -= above;
-    if (cnt_d == need) {
-      take_all = true;
-      break;
-    }
-  }
-  __syncthreads();
-}
-
-// Selected candidates in ascending index order: calls emit(j, position) for each of the k
-// selected j (position in [0, k)).  Ties at the threshold go to the lowest indices.
-template <int NT, typename Emit>
-__device__ void emit_topk(const uint32_t* keys, int m, uint32_t prefix, uint32_t mask, int need,
-                          bool take_all, int* scratch, Emit emit) {
-  const int tid = threadIdx.x;
-  const int per = (m + NT - 1) / NT;
-  const int j0 = min(m, tid * per), j1 = min(m, j0 + per);
-  int eq = 0;
-  for (int j = j0; j < j1; ++j) eq += ((keys[j] & mask) == prefix);
-  int eq_rank = block_exclusive_scan<NT>(eq, scratch);
-  int cnt = 0;
-  {
-    int r = eq_rank;
-    for (int j = j0; j < j1; ++j) {
-      const uint32_t km = keys[j] & mask;
-      const bool is_eq = km == prefix;
-      cnt += (km > prefix) || (is_eq && (take_all || r < need));
-      r += is_eq;
-    }
-  }
-  int pos = block_exclusive_scan<NT>(cnt, scratch);
-  int r = eq_rank;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t km = keys[j] & mask;
-    const bool is_eq = km == prefix;
-    if ((km > prefix) || (is_eq && (take_all || r < need))) emit(j, pos++);
-    r += is_eq;
-  }
-}
-
 // ---- online-softmax state merge (base-2 exponent) --------------------------------------
 __device__ __forceinline__ void merge_scale(float ma, float mb, float& M, float& fa, float& fb) {
   M = fmaxf(ma, mb);
@@ -213,6 +90,11 @@ __device__ __forceinline__ void cp_async_commit() {
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;\n" ::: "memory");
 }
+// Wait until at most N of this thread's committed cp.async groups are still pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
@@ -235,6 +117,70 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
       "{%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+}  // namespace vt
+
+namespace vt {
+
+// ---- mbarrier + bulk async copies (TMA engine, no multicast) ----------------------------
+// Device status bit: an mbarrier wait gave up (a copy never landed); the CTA skipped its work.
+constexpr int kDevTimeout = 16;
+// A wait gives up after this many nanoseconds of the global timer (copies from HBM land in
+// microseconds; only a broken byte count could exhaust it).
+constexpr unsigned long long kWaitNs = 200ull * 1000 * 1000;
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+// Make barrier initialisation visible to the async proxy (the copy engine).
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+// Order this thread's earlier generic-proxy shared-memory accesses before later bulk copies
+// into the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+// Bounded wait for the phase with the given parity; false if it did not complete in time.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitNs) return false;
+  }
+}
+// One contiguous global -> shared copy of `bytes` (multiple of 16, both ends 16-byte aligned)
+// that signals `bar` with its byte count when it lands.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
 }  // namespace vt

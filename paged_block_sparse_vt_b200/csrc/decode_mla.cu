@@ -21,6 +21,7 @@
 // of the request) and serve as both the K operand and, through a transposed ldmatrix, the
 // V operand.
 #include "decode_params.cuh"
+#include "topk.cuh"
 
 namespace vt {
 
@@ -43,7 +44,7 @@ __host__ __device__ inline MlaSmem mla_smem_layout(int G, int cand_cap, int key_
   int o = 0;
   s.sel = o;  o += align16(kmax * 4);
   s.phys = o; o += align16(kmax * 4);
-  s.misc = o; o += align16(320 * 4);
+  s.misc = o; o += align16((kTopkBins + 64) * 4);
   const int base = o;
   int a = base;  // selection phase
   s.qm = a;    a += align16(kMlaD * 4);
@@ -82,10 +83,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const Decode
   const MlaSmem Ls = mla_smem_layout(G, p.cand_cap, p.key_cap, p.kmax, ppc);
   int* s_sel = reinterpret_cast<int*>(smem + Ls.sel);
   int* s_phys = reinterpret_cast<int*>(smem + Ls.phys);
-  int* s_misc = reinterpret_cast<int*>(smem + Ls.misc);
-  int* s_hist = s_misc;
-  int* s_info = s_misc + 256;
-  int* s_scan = s_misc + 264;
+  int* s_hist = reinterpret_cast<int*>(smem + Ls.misc);  // kTopkBins
+  int* s_small = s_hist + kTopkBins;                      // 64
 
   const int bslot = blockIdx.x / C;  // Hkv == 1: one unit per request
   const int b = p.order ? p.order[bslot] : bslot;
@@ -209,19 +208,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const Decode
         for (int j = tid; j < p.bos; j += NT) s_sel[j] = j;
         for (int j = tid; j < p.eos; j += NT) s_sel[p.bos + p.topk + j] = n - p.eos + j;
         __syncthreads();
-        if (p.topk > 0) {
-          uint32_t prefix, mask;
-          int need;
-          bool take_all;
-          radix_select<NT>(s_key, m, p.topk, s_hist, s_info, prefix, mask, need, take_all);
-          const int bos = p.bos, topk = p.topk;
-          emit_topk<NT>(s_key, m, prefix, mask, need, take_all, s_scan, [&](int j, int pos) {
-            if (pos < topk) s_sel[bos + pos] = bos + j;  // exactly topk emitted; guard anyway
-          });
-        }
+        const int bos = p.bos, topk = p.topk;
+        block_topk<NT>(s_key, m, topk, s_hist, s_small, [&](int j, int pos) {
+          if (pos < topk) s_sel[bos + pos] = bos + j;  // exactly topk are emitted
+        });
       }
       cluster.sync();  // #2
-      if (rank != 0) {
+      // Only the attending modes need the selection in every CTA.  In kSelect mode rank 0
+      // returns right after writing it out, so nobody may touch its shared memory here.
+      if (MODE != kSelect && rank != 0) {
         const int* r0sel = cluster.map_shared_rank(s_sel, 0);
         for (int j = tid; j < ns; j += NT) s_sel[j] = r0sel[j];
       }
@@ -419,12 +414,9 @@ static cudaError_t launch_mla_t(const DecodeParams& p, int C, cudaStream_t strea
   auto kern = mla_decode_kernel<G, MODE>;
   const int ppc = (p.kmax + C - 1) / C;
   const MlaSmem L = mla_smem_layout(G, p.cand_cap, p.key_cap, p.kmax, ppc);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+  static std::atomic<int> optin[64];
+  cudaError_t e = ensure_smem_optin(kern, L.total, C > 8, optin);
   if (e != cudaSuccess) return e;
-  if (C > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((int64_t)C * p.B), 1, 1);
   cfg.blockDim = dim3(kMlaThreads, 1, 1);

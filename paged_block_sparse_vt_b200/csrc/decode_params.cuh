@@ -39,26 +39,40 @@ struct DecodeParams {
 
 __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 
-// Shared-memory carve-up of the CUDA-core decode kernel (byte offsets).
-struct FmaSmem {
-  int qm, cpage, score, key, sel, phys, warp, cta, misc, total;
+// Shared-memory carve-up of the GQA decode kernel (byte offsets).
+struct GqaSmem {
+  int score, sel, phys, qm, cpage, key, misc, ring, warp, cta, total;
 };
 
-__host__ __device__ inline FmaSmem fma_smem_layout(int D, int G, int NW, int cand_cap, int key_cap,
-                                                   int kmax) {
-  FmaSmem s;
-  int o = 0;
-  s.qm = o;    o += align16(D * 4);
-  s.cpage = o; o += align16(cand_cap * 4);
-  s.score = o; o += align16(cand_cap * 4);
-  s.key = o;   o += align16(key_cap * 4);
-  s.sel = o;   o += align16(kmax * 4);
-  s.phys = o;  o += align16(kmax * 4);
-  s.warp = o;  o += align16(NW * G * (D + 2) * 4);
-  s.cta = o;   o += align16(G * (D + 2) * 4);
-  s.misc = o;  o += align16(320 * 4);
-  s.total = o;
-  return s;
+}  // namespace vt
+
+#include <atomic>
+
+namespace vt {
+
+// cudaFuncSetAttribute once per (kernel, device) and size: the shared-memory opt-in only
+// ever grows, so a later call asking for no more than what was set makes no runtime call
+// (which also keeps repeated launches cheap on the host and safe inside stream capture).
+// `cache` is a per-kernel array indexed by device: bytes * 2 + (non-portable cluster bit).
+template <typename Kernel>
+inline cudaError_t ensure_smem_optin(Kernel kern, int bytes, bool nonportable_cluster,
+                                     std::atomic<int>* cache) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::atomic<int>& slot = cache[dev & 63];
+  const int have = slot.load(std::memory_order_acquire);
+  if (have != 0 && (have >> 1) >= bytes && (!nonportable_cluster || (have & 1))) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (nonportable_cluster) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  const int hb = have >> 1;
+  slot.store(((hb > bytes ? hb : bytes) << 1) | (have & 1) | (nonportable_cluster ? 1 : 0),
+             std::memory_order_release);
+  return cudaSuccess;
 }
 
 }  // namespace vt
