@@ -4,9 +4,11 @@ One step = one decode layer of the Qwen3-0.6B-like workload (B=32, Hq=16, Hkv=8,
 page 16, contexts U[4096, 16384], 40,000-page shuffled pool, top-30 + 1 + 1 pages):
   vt_build_centroids  on the pages that fill at this step (requests whose length is a
                       multiple of 16),
-  vt_plan_requests    request order, longest first,
   vt_sparse_decode_fused  group mean -> centroid scores -> exact top-k + reserved pages ->
-                      attention over the selected pages, one launch.
+                      attention over the selected pages, one launch of persistent CTAs
+                      that schedule themselves (``--plan`` adds vt_plan_requests, the
+                      longest-first order the cluster kernels take; the persistent kernel
+                      does not need it).
 Inputs are resident in HBM; steps rotate over ``--replicas`` copies of the inputs (pools,
 centroids, q, page tables) whose combined footprint is far above the 126 MB L2, so no step
 finds its data in L2.  Rank 0 prints one JSON line.
@@ -87,9 +89,14 @@ def read_peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# the files the timed fused kernel is compiled from
+FUSED_KERNEL_SOURCES = ("fused_persistent.cu", "gqa_attend.cuh", "topk.cuh", "common.cuh",
+                        "decode_params.cuh")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("decode_fma.cu", "common.cuh", "decode_params.cuh"):
+    for name in FUSED_KERNEL_SOURCES:
         with open(os.path.join(ROOT, "paged_block_sparse_vt_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -312,6 +319,8 @@ def run_ours(args, world, rank, local):
         d["lse"] = torch.empty((c.B, c.Hq), dtype=torch.float32, device=dev)
         d["order"] = torch.empty((c.B,), dtype=torch.int32, device=dev)
         d["status"] = torch.zeros((1,), dtype=torch.int32, device=dev)
+        d["ws"] = vt.fused_workspace(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                     d["seq_lens"], d["cent"], c.topk, c.bos, c.eos)
         reps.append(d)
     torch.cuda.synchronize(dev)
 
@@ -319,15 +328,16 @@ def run_ours(args, world, rank, local):
         vt.vt_sparse_decode_fused(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
                                   d["seq_lens"], d["cent"], c.topk, c.bos, c.eos, c.sm_scale,
                                   out=d["out"], lse=d["lse"],
-                                  order=None if args.no_plan else d["order"], status=d["status"])
+                                  order=d["order"] if args.plan else None, status=d["status"],
+                                  workspace=d["ws"])
 
     def step(d):
         vt.vt_build_centroids(d["k_pool"], d["fill_pages"], d["cent"], status=d["status"])
-        if not args.no_plan:
+        if args.plan:
             vt.vt_plan_requests(d["seq_lens"], d["order"])
         fused(d)
 
-    launches_per_step = 2 + (0 if args.no_plan else 1)
+    launches_per_step = 2 + (1 if args.plan else 0)
     for i in range(args.warmup):
         step(reps[i % args.replicas])
     torch.cuda.synchronize(dev)
@@ -417,7 +427,7 @@ def run_ours(args, world, rank, local):
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "traffic": recorded_traffic(),
-            "kernel": "fma_decode_kernel (vt_sparse_decode_fused)",
+            "kernel": "persist_fused_kernel (vt_sparse_decode_fused)",
             "algorithmic_bytes_per_launch": nbytes["fused"], "kernel_ms": fused_ms,
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
             else "fallback 6650 GB/s",
@@ -463,7 +473,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--replicas", type=int, default=3)
-    ap.add_argument("--no-plan", action="store_true", help="skip the planner launch")
+    ap.add_argument("--plan", action="store_true",
+                    help="add the vt_plan_requests launch to the step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

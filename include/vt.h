@@ -20,7 +20,8 @@
  *   - Every data pointer is DEVICE memory owned by the caller.  The library
  *     never allocates, frees or synchronises; each call enqueues its kernels
  *     on `stream` (a cudaStream_t passed as void*; NULL = legacy default
- *     stream) and returns.  No workspace is needed.
+ *     stream) and returns.  Only vt_sparse_decode_fused takes a workspace
+ *     (see vt_fused_workspace_size).
  *   - bf16 means IEEE bfloat16 (upper half of a binary32), fp32 is binary32.
  *   - Host-side argument checks fail fast with VT_ERR_INVALID_ARG or
  *     VT_ERR_UNSUPPORTED before anything is launched; a failed launch returns
@@ -61,6 +62,8 @@ typedef enum {
 #define VT_DEV_BAD_PAGE 1 /* a page id outside [0, num_pages); that unit/page was skipped */
 #define VT_DEV_BAD_LEN 2  /* seq_len < 1, or ceil(seq_len/16) > pt_stride; unit skipped */
 #define VT_DEV_BAD_SEL 4  /* n_sel or a sel entry out of range (vt_sparse_decode); unit skipped */
+#define VT_DEV_BAD_ORDER 8 /* an `order` entry outside [0, B); that request slot was skipped */
+#define VT_DEV_TIMEOUT 16  /* a wait for work published by another CTA gave up (never expected) */
 
 /*
  * Paged K/V layout ("vTensor" metadata, reduced to one descriptor).
@@ -151,13 +154,35 @@ vt_status vt_sparse_decode(const vt_paged_kv* kv, const vt_decode_args* a, const
                            const int32_t* n_sel, void* out, float* lse, void* stream);
 
 /*
- * The whole query side in one launch (selection + attention, "kernel fusion
- * ... to minimize memory traffic", rndamp.com article, same section).  Same
- * results as vt_select_pages followed by vt_sparse_decode.  sel / n_sel
+ * The whole query side in one call: selection + attention ("kernel fusion",
+ * and "a workload planner for balanced GPU scheduling", rndamp.com article,
+ * same section).  Same results as vt_select_pages followed by
+ * vt_sparse_decode up to fp32 rounding (and, where two candidate pages score
+ * within that rounding of each other, which of them is kept).  sel / n_sel
  * receive the selection when not NULL (both or neither).
+ *
+ * For GQA heads with B <= 2048 the work runs as one launch of persistent
+ * CTAs fed from a queue of small scan and attention items (after a one-CTA
+ * planner launch), which keeps every SM busy on batches of very uneven
+ * lengths; it needs `workspace`: device memory of vt_fused_workspace_size()
+ * bytes, 256-byte aligned, ZERO-FILLED ONCE when allocated.  Every call
+ * leaves it ready for the next one, so it is zeroed only once, but calls that
+ * share a workspace must not overlap on the GPU (use one stream, or one
+ * workspace per stream); after a call that reported VT_DEV_TIMEOUT, zero it
+ * again.  When vt_fused_workspace_size() is 0 (MLA, or B > 2048) no
+ * workspace is used and `workspace` may be NULL.
  */
 vt_status vt_sparse_decode_fused(const vt_paged_kv* kv, const vt_decode_args* a, void* out,
-                                 float* lse, int32_t* sel, int32_t* n_sel, void* stream);
+                                 float* lse, int32_t* sel, int32_t* n_sel, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
+ * Bytes of workspace vt_sparse_decode_fused needs for these arguments (0 if
+ * none); depends only on the shapes (B, Hq, Hkv, head dims, pt_stride, topk,
+ * bos, eos), not on the data.  Returns 0 as well for arguments that
+ * vt_sparse_decode_fused would reject.
+ */
+size_t vt_fused_workspace_size(const vt_paged_kv* kv, const vt_decode_args* a);
 
 /*
  * Workload planner ("a workload planner for balanced GPU scheduling", same

@@ -12,10 +12,13 @@ from .binding import (  # noqa: F401
     VT_DEV_BAD_ORDER,
     VT_DEV_BAD_PAGE,
     VT_DEV_BAD_SEL,
+    VT_DEV_TIMEOUT,
     VtError,
+    fused_workspace,
     load_library,
     vt_abi_version,
     vt_build_centroids,
+    vt_fused_workspace_size,
     vt_plan_requests,
     vt_select_pages,
     vt_sparse_decode,

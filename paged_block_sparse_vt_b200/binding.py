@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libvt.so")
 
 VT_OK, VT_ERR_INVALID_ARG, VT_ERR_UNSUPPORTED, VT_ERR_CUDA = 0, 1, 2, 3
-VT_DEV_BAD_PAGE, VT_DEV_BAD_LEN, VT_DEV_BAD_SEL, VT_DEV_BAD_ORDER = 1, 2, 4, 8
+VT_DEV_BAD_PAGE, VT_DEV_BAD_LEN, VT_DEV_BAD_SEL, VT_DEV_BAD_ORDER, VT_DEV_TIMEOUT = 1, 2, 4, 8, 16
 PAGE_SIZE = 16
 
 
@@ -51,7 +51,8 @@ class DecodeArgs(ctypes.Structure):
 
 
 EXPORTS = ("vt_build_centroids", "vt_select_pages", "vt_sparse_decode", "vt_sparse_decode_fused",
-           "vt_plan_requests", "vt_status_string", "vt_last_error_detail", "vt_abi_version")
+           "vt_fused_workspace_size", "vt_plan_requests", "vt_status_string",
+           "vt_last_error_detail", "vt_abi_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -72,13 +73,15 @@ def load_library(path: str = LIB_PATH):
                 "vt_build_centroids": [kv, P, I32, P, P, P],
                 "vt_select_pages": [kv, args, P, P, P],
                 "vt_sparse_decode": [kv, args, P, P, P, P, P],
-                "vt_sparse_decode_fused": [kv, args, P, P, P, P, P],
+                "vt_sparse_decode_fused": [kv, args, P, P, P, P, P, ctypes.c_size_t, P],
                 "vt_plan_requests": [P, I32, P, P],
             }
             for name, argtypes in sigs.items():
                 fn = getattr(lib, name)
                 fn.argtypes = argtypes
                 fn.restype = ctypes.c_int
+            lib.vt_fused_workspace_size.argtypes = [kv, args]
+            lib.vt_fused_workspace_size.restype = ctypes.c_size_t
             lib.vt_status_string.argtypes = [ctypes.c_int]
             lib.vt_status_string.restype = ctypes.c_char_p
             lib.vt_last_error_detail.argtypes = []
@@ -200,10 +203,34 @@ def vt_sparse_decode(q, k_pool, v_pool, page_table, seq_lens, sel, n_sel, sm_sca
     return out, lse
 
 
+def vt_fused_workspace_size(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos, eos,
+                            head_dim_v=None) -> int:
+    """Bytes of workspace vt_sparse_decode_fused needs for these shapes (0 if none)."""
+    lib = load_library()
+    kv = paged_kv(k_pool, v_pool, head_dim_v)
+    a = decode_args(q, page_table, seq_lens, centroids, topk, bos, eos, 1.0)
+    return int(lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(a)))
+
+
+def fused_workspace(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos, eos,
+                    head_dim_v=None) -> Optional[torch.Tensor]:
+    """A zero-filled workspace for vt_sparse_decode_fused (None when none is needed).
+
+    Zero it once; every call leaves it ready for the next.  Calls sharing one workspace must
+    not overlap on the GPU.
+    """
+    n = vt_fused_workspace_size(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos,
+                                eos, head_dim_v)
+    return torch.zeros(n, dtype=torch.uint8, device=q.device) if n else None
+
+
 def vt_sparse_decode_fused(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos, eos,
                            sm_scale, out=None, lse=None, sel=None, n_sel=None, order=None,
-                           status=None, head_dim_v=None, want_lse=True):
-    """Selection + attention in one launch.  Returns (out, lse, sel, n_sel)."""
+                           status=None, head_dim_v=None, want_lse=True, workspace=None):
+    """Selection + attention in one call.  Returns (out, lse, sel, n_sel).
+
+    ``workspace``: from fused_workspace(); allocated (zeroed) here when not given.
+    """
     lib = load_library()
     kv = paged_kv(k_pool, v_pool, head_dim_v)
     a = decode_args(q, page_table, seq_lens, centroids, topk, bos, eos, sm_scale, order, status)
@@ -212,8 +239,14 @@ def vt_sparse_decode_fused(q, k_pool, v_pool, page_table, seq_lens, centroids, t
         out = torch.empty((B, hq, kv.head_dim_v), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = int(lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(a)))
+        workspace = torch.zeros(n, dtype=torch.uint8, device=q.device) if n else None
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8, contiguous=True)
     rc = lib.vt_sparse_decode_fused(ctypes.byref(kv), ctypes.byref(a), out.data_ptr(), _ptr(lse),
-                                    _ptr(sel), _ptr(n_sel), _stream(q))
+                                    _ptr(sel), _ptr(n_sel), _ptr(workspace),
+                                    0 if workspace is None else workspace.numel(), _stream(q))
     _check(rc, "vt_sparse_decode_fused")
     return out, lse, sel, n_sel
 

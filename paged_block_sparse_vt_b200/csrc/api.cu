@@ -17,6 +17,11 @@ cudaError_t launch_mla_decode(const DecodeParams& p, int mode, int G, int C, cud
 int mla_smem_bytes(int G, int cand_cap, int key_cap, int kmax, int pages_per_cta);
 int mla_max_pages_per_cta();
 cudaError_t launch_plan(const int32_t* seq_lens, int B, int32_t* order, cudaStream_t s);
+size_t persist_workspace_bytes(const DecodeParams& p, int G, int Dv);
+int persist_smem_bytes(const DecodeParams& p, int D, int G);
+int persist_max_batch();
+cudaError_t launch_persist_fused(const DecodeParams& p, int D, int G, void* ws, int sm_count,
+                                 cudaStream_t s);
 }  // namespace vt
 
 using namespace vt;
@@ -184,8 +189,14 @@ vt_status fill_params(const vt_paged_kv* kv, const vt_decode_args* a, bool need_
   return ok();
 }
 
+// The fused GQA call runs on persistent CTAs (needs a workspace) up to this many requests.
+bool use_persistent(const Shape& sh, const vt_decode_args* a) {
+  return sh.path == kPathGqa && a->batch >= 1 && a->batch <= persist_max_batch();
+}
+
 vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int mode,
-                            int32_t* sel, int32_t* n_sel, void* out, float* lse, void* stream) {
+                            int32_t* sel, int32_t* n_sel, void* out, float* lse, void* ws,
+                            size_t ws_bytes, void* stream) {
   Shape sh;
   DecodeParams p;
   vt_status s = fill_params(kv, a, mode != kDecode, &sh, &p);
@@ -200,12 +211,25 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
   p.n_sel = n_sel;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mode == kFused && use_persistent(sh, a)) {
+    const size_t need = persist_workspace_bytes(p, sh.G, sh.Dv);
+    if (!ws || ws_bytes < need)
+      return fail(VT_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need,
+                  ws ? ws_bytes : (size_t)0);
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+      return fail(VT_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+    const int bytes = persist_smem_bytes(p, sh.D, sh.G);
+    if (bytes > 227 * 1024) return fail(VT_ERR_UNSUPPORTED, "shared memory need %d B too large", bytes);
+    cudaError_t e = launch_persist_fused(p, sh.D, sh.G, ws, sm_count(), st);
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return ok();
+  }
   const int64_t units = (int64_t)a->batch * kv->num_kv_heads;
   const int C = pick_cluster(sh, units, p.kmax);
   const int max_cand = (int)std::max<int64_t>(1, a->pt_stride - a->bos - a->eos);
   p.key_cap = max_cand;
   p.cand_cap = (max_cand + C - 1) / C;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (sh.path == kPathGqa) {
     const int bytes = gqa_smem_bytes(sh.D, sh.G, p.cand_cap, p.key_cap, p.kmax);
@@ -246,18 +270,28 @@ vt_status vt_build_centroids(const vt_paged_kv* kv, const int32_t* pages, int32_
 
 vt_status vt_select_pages(const vt_paged_kv* kv, const vt_decode_args* a, int32_t* sel,
                           int32_t* n_sel, void* stream) {
-  return launch_query_side(kv, a, kSelect, sel, n_sel, nullptr, nullptr, stream);
+  return launch_query_side(kv, a, kSelect, sel, n_sel, nullptr, nullptr, nullptr, 0, stream);
 }
 
 vt_status vt_sparse_decode(const vt_paged_kv* kv, const vt_decode_args* a, const int32_t* sel,
                            const int32_t* n_sel, void* out, float* lse, void* stream) {
   return launch_query_side(kv, a, kDecode, const_cast<int32_t*>(sel),
-                           const_cast<int32_t*>(n_sel), out, lse, stream);
+                           const_cast<int32_t*>(n_sel), out, lse, nullptr, 0, stream);
 }
 
 vt_status vt_sparse_decode_fused(const vt_paged_kv* kv, const vt_decode_args* a, void* out,
-                                 float* lse, int32_t* sel, int32_t* n_sel, void* stream) {
-  return launch_query_side(kv, a, kFused, sel, n_sel, out, lse, stream);
+                                 float* lse, int32_t* sel, int32_t* n_sel, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  return launch_query_side(kv, a, kFused, sel, n_sel, out, lse, workspace, workspace_bytes,
+                           stream);
+}
+
+size_t vt_fused_workspace_size(const vt_paged_kv* kv, const vt_decode_args* a) {
+  Shape sh;
+  DecodeParams p;
+  if (fill_params(kv, a, true, &sh, &p) != VT_OK) return 0;
+  if (!use_persistent(sh, a)) return 0;
+  return persist_workspace_bytes(p, sh.G, sh.Dv);
 }
 
 vt_status vt_plan_requests(const int32_t* seq_lens, int32_t batch, int32_t* order, void* stream) {

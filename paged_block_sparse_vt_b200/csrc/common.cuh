@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/vt.h"
+#include "vt.h"  // include/ is on the include path
 
 namespace vt {
 
@@ -17,8 +17,7 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// Extra device status bit: an `order` entry outside [0, B).
-constexpr int kDevBadOrder = 8;
+constexpr int kDevBadOrder = VT_DEV_BAD_ORDER;
 
 // ---- bf16 <-> fp32 -------------------------------------------------------------------
 // A bf16 value is the upper half of a binary32: widening is a 16-bit shift.
@@ -123,64 +122,16 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
 
 namespace vt {
 
-// ---- mbarrier + bulk async copies (TMA engine, no multicast) ----------------------------
-// Device status bit: an mbarrier wait gave up (a copy never landed); the CTA skipped its work.
-constexpr int kDevTimeout = 16;
-// A wait gives up after this many nanoseconds of the global timer (copies from HBM land in
-// microseconds; only a broken byte count could exhaust it).
+// ---- bounded waits -----------------------------------------------------------------------
+constexpr int kDevTimeout = VT_DEV_TIMEOUT;
+// A wait gives up after this many nanoseconds of the global timer (everything waited for is
+// produced within microseconds; only a bug could exhaust it).
 constexpr unsigned long long kWaitNs = 200ull * 1000 * 1000;
 
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
   return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
-}
-// Make barrier initialisation visible to the async proxy (the copy engine).
-__device__ __forceinline__ void mbar_init_fence() {
-  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-}
-// Order this thread's earlier generic-proxy shared-memory accesses before later bulk copies
-// into the same bytes.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-// Bounded wait for the phase with the given parity; false if it did not complete in time.
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(done)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  for (;;) {
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitNs) return false;
-  }
-}
-// One contiguous global -> shared copy of `bytes` (multiple of 16, both ends 16-byte aligned)
-// that signals `bar` with its byte count when it lands.
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
-                                         uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::
-          "r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
 }
 
 }  // namespace vt

@@ -31,6 +31,7 @@
 //      DSMEM, each CTA writing 1/C of the unit's G x D outputs (and lse).
 // A request with n <= topk+bos+eos pages skips 1-2 and attends to every page.
 #include "decode_params.cuh"
+#include "gqa_attend.cuh"
 #include "topk.cuh"
 
 namespace vt {
@@ -41,17 +42,11 @@ constexpr int kGqaSlots = 3;       // page slots per warp: one computing, two la
 constexpr int kScanSlots = 6;      // centroid batches (8 rows) per warp: five landing
 
 template <int D>
-struct GqaShape {
-  static constexpr int ROW = D + 8;            // smem row stride in elements (conflict-free ldmatrix)
-  static constexpr int TILE = kPage * ROW * 2;  // bytes of one K or V page tile
-  static constexpr int SLOT = 2 * TILE;         // K tile, then V tile
-  static constexpr int KS = D / 16;             // k-steps of S = Q K^T
-  static constexpr int NT = D / 8;              // n-tiles of O = P V
-  static constexpr int CPR = D / 8;             // 16-byte chunks per K/V row
+struct GqaShape : PageTile<D> {
   static constexpr int C_ROW = D * 4;           // bytes of one fp32 centroid row
   static constexpr int SCAN_SLOT = 8 * C_ROW;   // one batch: 8 centroid rows
-  static constexpr int WARP_RING = (kGqaSlots * SLOT > kScanSlots * SCAN_SLOT)
-                                       ? kGqaSlots * SLOT : kScanSlots * SCAN_SLOT;
+  static constexpr int WARP_RING = (kGqaSlots * PageTile<D>::SLOT > kScanSlots * SCAN_SLOT)
+                                       ? kGqaSlots * PageTile<D>::SLOT : kScanSlots * SCAN_SLOT;
 };
 
 __host__ __device__ inline GqaSmem gqa_smem_layout(int D, int G, int cand_cap, int key_cap,
@@ -82,14 +77,6 @@ __host__ __device__ inline GqaSmem gqa_smem_layout(int D, int G, int cand_cap, i
   return s;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  const uint32_t l = (uint32_t)__bfloat16_as_ushort(__float2bfloat16(lo));
-  const uint32_t h = (uint32_t)__bfloat16_as_ushort(__float2bfloat16(hi));
-  return l | (h << 16);
-}
-__device__ __forceinline__ float bf16_round(float x) {
-  return __bfloat162float(__float2bfloat16(x));
-}
 template <int D, int G, int MODE>
 __global__ void __launch_bounds__(kGqaThreads) gqa_decode_kernel(const DecodeParams p) {
   using S = GqaShape<D>;
@@ -289,139 +276,36 @@ __global__ void __launch_bounds__(kGqaThreads) gqa_decode_kernel(const DecodePar
 
   // one page (16 K rows and 16 V rows of head h) into slot i % kGqaSlots; rows past the end
   // of the request (or of an unusable page) are zero-filled instead of read
+  auto rows_of = [&](int j) { return s_phys[j] < 0 ? 0 : (s_sel[j] == n - 1 ? last_valid : kPage); };
   auto issue = [&](int i) {
     if (i < npw) {
       const int j = j0 + warp + NW * i;
-      const int pg = s_phys[j];
-      const int vr = pg < 0 ? 0 : (s_sel[j] == n - 1 ? last_valid : kPage);
-      const __nv_bfloat16* kp = p.k_pool + (int64_t)(pg < 0 ? 0 : pg) * p.sk_p + (int64_t)h * p.sk_h;
-      const __nv_bfloat16* vp = p.v_pool + (int64_t)(pg < 0 ? 0 : pg) * p.sv_p + (int64_t)h * p.sv_h;
-      const uint32_t dst = ring + (i % kGqaSlots) * S::SLOT;
-      constexpr int RPI = 32 / S::CPR;  // rows per warp instruction
-#pragma unroll
-      for (int t = 0; t < kPage / RPI; ++t) {
-        const int row = t * RPI + lane / S::CPR, k = lane % S::CPR;
-        const bool ok = row < vr;
-        const uint32_t o = (row * S::ROW + k * 8) * 2;
-        cp_async16(dst + o, ok ? kp + (int64_t)row * p.sk_t + k * 8 : p.k_pool, ok ? 16 : 0);
-        cp_async16(dst + S::TILE + o, ok ? vp + (int64_t)row * p.sv_t + k * 8 : p.v_pool,
-                   ok ? 16 : 0);
-      }
+      const int64_t pg = s_phys[j] < 0 ? 0 : s_phys[j];
+      stage_page<D>(ring + (i % kGqaSlots) * S::SLOT, p.k_pool + pg * p.sk_p + (int64_t)h * p.sk_h,
+                    p.v_pool + pg * p.sv_p + (int64_t)h * p.sv_h, p.sk_t, p.sv_t, rows_of(j),
+                    p.k_pool, lane);
     }
     cp_async_commit();
   };
 #pragma unroll
   for (int i = 0; i < kGqaSlots - 1; ++i) issue(i);
-
-  // Q as the A operand (rows = query heads g = lane / 4, rows >= G and 8..15 are zero)
-  const int g = lane >> 2, qd = 2 * (lane & 3);
-  uint32_t qa0[S::KS], qa2[S::KS];
-#pragma unroll
-  for (int ks = 0; ks < S::KS; ++ks) {
-    if (g < G) {
-      const __nv_bfloat16* qrow = p.q + (orow + g) * D + ks * 16 + qd;
-      qa0[ks] = *reinterpret_cast<const uint32_t*>(qrow);
-      qa2[ks] = *reinterpret_cast<const uint32_t*>(qrow + 8);
-    } else {
-      qa0[ks] = qa2[ks] = 0u;
-    }
-  }
-  float o[S::NT][4];
-#pragma unroll
-  for (int t = 0; t < S::NT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.0f;
-  float mrun = -INFINITY, lrun = 0.0f;  // running max / partial sum of head g (this lane)
-  const uint32_t koff = (((lane & 7) + ((lane >> 4) << 3)) * S::ROW + ((lane >> 3) & 1) * 8) * 2;
-  const uint32_t voff = (((lane & 7) + ((lane >> 3) & 1) * 8) * S::ROW + (lane >> 4) * 8) * 2;
-
+  WarpAttention<D, G> att;
+  att.init(p.q + orow * D, lane);
   for (int i = 0; i < npw; ++i) {
     issue(i + kGqaSlots - 1);
     cp_async_wait<kGqaSlots - 1>();
     __syncwarp();  // page i is in this warp's slot for every lane
-    const int j = j0 + warp + NW * i;
-    const int vr = s_phys[j] < 0 ? 0 : (s_sel[j] == n - 1 ? last_valid : kPage);
-    const uint32_t kt = ring + (i % kGqaSlots) * S::SLOT, vt = kt + S::TILE;
-    // S = Q K^T for the 16 tokens (two n-tiles of 8)
-    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < S::KS; ++ks) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(kt + koff + ks * 32, b0, b1, b2, b3);
-      mma_16816(s0, qa0[ks], 0u, qa2[ks], 0u, b0, b1);
-      mma_16816(s1, qa0[ks], 0u, qa2[ks], 0u, b2, b3);
-    }
-    // this lane holds head g at tokens qd, qd+1 (s0) and 8+qd, 9+qd (s1)
-    const bool live = g < G;
-    float z0 = (live && qd < vr) ? s0[0] * p.qscale : -INFINITY;
-    float z1 = (live && qd + 1 < vr) ? s0[1] * p.qscale : -INFINITY;
-    float z2 = (live && qd + 8 < vr) ? s1[0] * p.qscale : -INFINITY;
-    float z3 = (live && qd + 9 < vr) ? s1[1] * p.qscale : -INFINITY;
-    float mx = fmaxf(fmaxf(z0, z1), fmaxf(z2, z3));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-    const float mnew = fmaxf(mrun, mx);
-    const float corr = (mnew == -INFINITY) ? 1.0f : exp2f(mrun - mnew);
-    // probabilities rounded to bf16 once: the same values feed the MMA and the sum
-    const float p0 = z0 == -INFINITY ? 0.0f : bf16_round(exp2f(z0 - mnew));
-    const float p1 = z1 == -INFINITY ? 0.0f : bf16_round(exp2f(z1 - mnew));
-    const float p2 = z2 == -INFINITY ? 0.0f : bf16_round(exp2f(z2 - mnew));
-    const float p3 = z3 == -INFINITY ? 0.0f : bf16_round(exp2f(z3 - mnew));
-    lrun = lrun * corr + ((p0 + p1) + (p2 + p3));
-    mrun = mnew;
-#pragma unroll
-    for (int t = 0; t < S::NT; ++t) {
-      o[t][0] *= corr;
-      o[t][1] *= corr;
-    }
-    const uint32_t pa0 = pack_bf16(p0, p1), pa2 = pack_bf16(p2, p3);
-    // O += P V over the page's 16 tokens, two n-tiles of 8 dims per ldmatrix
-#pragma unroll
-    for (int n2 = 0; n2 < S::NT / 2; ++n2) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(vt + voff + n2 * 32, b0, b1, b2, b3);
-      mma_16816(o[2 * n2], pa0, 0u, pa2, 0u, b0, b1);
-      mma_16816(o[2 * n2 + 1], pa0, 0u, pa2, 0u, b2, b3);
-    }
+    att.page(ring + (i % kGqaSlots) * S::SLOT, rows_of(j0 + warp + NW * i), p.qscale);
     __syncwarp();  // every lane is done with slot i before a later issue refills it
   }
   cp_async_wait<0>();
-  lrun += __shfl_xor_sync(kFull, lrun, 1);
-  lrun += __shfl_xor_sync(kFull, lrun, 2);
   __syncthreads();  // all warps are out of their slots: the combine area may reuse them
 
   float* s_warp = reinterpret_cast<float*>(smem + Ls.warp);  // [NW][G][D+2]: acc, m, l
   float* s_cta = reinterpret_cast<float*>(smem + Ls.cta);    // [G][D+2]
-  if (g < G) {
-    float* w = s_warp + (warp * G + g) * (D + 2);
-#pragma unroll
-    for (int t = 0; t < S::NT; ++t) {
-      w[t * 8 + qd] = o[t][0];
-      w[t * 8 + qd + 1] = o[t][1];
-    }
-    if ((lane & 3) == 0) {
-      w[D] = mrun;
-      w[D + 1] = lrun;
-    }
-  }
+  att.store(s_warp + warp * G * (D + 2), lane);
   __syncthreads();
-  for (int idx = tid; idx < G * D; idx += NT) {
-    const int gg = idx / D, d = idx - gg * D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_warp[(w * G + gg) * (D + 2) + D]);
-    float A = 0.0f, Lsum = 0.0f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float* pw = s_warp + (w * G + gg) * (D + 2);
-      const float f = (pw[D] == -INFINITY) ? 0.0f : exp2f(pw[D] - M);
-      A = fmaf(pw[d], f, A);
-      Lsum = fmaf(pw[D + 1], f, Lsum);
-    }
-    s_cta[gg * (D + 2) + d] = A;
-    if (d == 0) {
-      s_cta[gg * (D + 2) + D] = M;
-      s_cta[gg * (D + 2) + D + 1] = Lsum;
-    }
-  }
+  merge_partials<G, D>(s_warp, NW, s_cta, tid, NT);
   cluster.sync();  // #2: every CTA's partial is visible (and every score has been read)
 
   // 4. each CTA finalises a 1/C slice of the unit's G x D outputs

@@ -27,7 +27,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     text = open(HEADER).read()
-    declared = set(re.findall(r"^\s*(?:vt_status|const char\*|int32_t)\s+(vt_\w+)\s*\(", text, re.M))
+    declared = set(re.findall(r"^\s*(?:vt_status|const char\*|int32_t|size_t)\s+(vt_\w+)\s*\(", text, re.M))
     assert declared == set(binding.EXPORTS)
     for name in declared:
         assert hasattr(lib, name), name
@@ -57,8 +57,10 @@ def _args(**over):
     return binding.DecodeArgs(**f)
 
 
-def _fused(lib, kv, a, out=FAKE + 0x600000, lse=None, sel=None, n_sel=None):
-    return lib.vt_sparse_decode_fused(ctypes.byref(kv), ctypes.byref(a), out, lse, sel, n_sel, None)
+def _fused(lib, kv, a, out=FAKE + 0x600000, lse=None, sel=None, n_sel=None, ws=FAKE + 0x8000000,
+           ws_bytes=1 << 40):
+    return lib.vt_sparse_decode_fused(ctypes.byref(kv), ctypes.byref(a), out, lse, sel, n_sel, ws,
+                                      ws_bytes, None)
 
 
 @pytest.mark.parametrize("kv_over,args_over,code", [
@@ -99,7 +101,7 @@ def test_fused_host_validation(lib, kv_over, args_over, code):
 def test_call_level_checks(lib):
     kv, a = _kv(), _args()
     assert lib.vt_sparse_decode_fused(ctypes.byref(kv), ctypes.byref(a), None, None, None, None,
-                                      None) == INV                       # out missing
+                                      FAKE, 1 << 40, None) == INV        # out missing
     assert _fused(lib, kv, a, sel=FAKE + 0x700000) == INV                # sel without n_sel
     assert lib.vt_select_pages(ctypes.byref(kv), ctypes.byref(a), None, FAKE, None) == INV
     assert lib.vt_sparse_decode(ctypes.byref(kv), ctypes.byref(a), FAKE, None, FAKE, None,
@@ -114,6 +116,24 @@ def test_call_level_checks(lib):
     assert lib.vt_plan_requests(FAKE, -2, FAKE, None) == INV
     assert lib.vt_plan_requests(FAKE, 0, FAKE, None) == OK
     assert lib.vt_plan_requests(None, 3, FAKE, None) == INV
+
+
+def test_fused_workspace_contract(lib):
+    kv, a = _kv(), _args()
+    need = lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(a))
+    assert need > 0 and need % 256 == 0
+    assert _fused(lib, kv, a, ws=None, ws_bytes=0) == INV                   # missing
+    assert _fused(lib, kv, a, ws=FAKE, ws_bytes=need - 1) == INV            # too small
+    assert _fused(lib, kv, a, ws=FAKE + 16, ws_bytes=need) == INV           # misaligned
+    # MLA and very large batches need none
+    mla = _kv(num_kv_heads=1, head_dim=576, head_dim_v=512, v_pool=FAKE, sk_h=576, sv_h=576,
+              sk_p=16 * 576, sv_p=16 * 576, sk_t=576, sv_t=576)
+    assert lib.vt_fused_workspace_size(ctypes.byref(mla), ctypes.byref(_args(num_q_heads=32))) == 0
+    assert lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(_args(batch=5000))) == 0
+    assert lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(_args(topk=-1))) == 0
+    # grows with the batch and with the chunks of the page-table row
+    assert lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(_args(batch=8))) > need
+    assert lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(_args(pt_stride=1024))) > need
 
 
 def test_binding_refuses_cpu_tensors():
