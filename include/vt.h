@@ -162,9 +162,9 @@ vt_status vt_sparse_decode(const vt_paged_kv* kv, const vt_decode_args* a, const
  * receive the selection when not NULL (both or neither).
  *
  * For GQA heads with B <= 2048 the work runs as one launch of persistent
- * CTAs fed from a queue of small scan and attention items (after a one-CTA
- * planner launch), which keeps every SM busy on batches of very uneven
- * lengths; it needs `workspace`: device memory of vt_fused_workspace_size()
+ * CTAs fed from a queue of small scan and attention items that the CTAs
+ * derive from seq_lens themselves (a->order is not used there), which keeps
+ * every SM busy on batches of very uneven lengths; it needs `workspace`: device memory of vt_fused_workspace_size()
  * bytes, 256-byte aligned, ZERO-FILLED ONCE when allocated.  Every call
  * leaves it ready for the next one, so it is zeroed only once, but calls that
  * share a workspace must not overlap on the GPU (use one stream, or one
