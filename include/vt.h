@@ -185,6 +185,38 @@ vt_status vt_sparse_decode_fused(const vt_paged_kv* kv, const vt_decode_args* a,
 size_t vt_fused_workspace_size(const vt_paged_kv* kv, const vt_decode_args* a);
 
 /*
+ * vt_sparse_decode_fused on a scratch buffer held inside the library instead
+ * of a caller-provided workspace, for callers that cannot allocate or keep
+ * one.  The method's pages have no counterpart to this call: it is a
+ * deployment convenience of this library.  Arguments, results and errors are
+ * those of vt_sparse_decode_fused without workspace / workspace_bytes.
+ *
+ * The scratch is one file-scope device array of VT_STATIC_SCRATCH_BYTES on
+ * each device the library is used on, placed and zero-filled by CUDA when the
+ * library's module is loaded there (the library itself never allocates).
+ * What must start at zero -- the work-queue and per-unit counters at the
+ * start of the scratch -- is zero at load, and every complete call leaves it
+ * zero again; the candidate and partial arrays after them are always written
+ * before they are read.  A call whose vt_fused_workspace_size() exceeds
+ * VT_STATIC_SCRATCH_BYTES fails with VT_ERR_UNSUPPORTED before anything is
+ * launched; shapes that need no workspace (MLA, B > 2048) run as
+ * vt_sparse_decode_fused does.
+ *
+ * Races: every call on one device shares the one scratch.  Two calls that can
+ * be on the GPU at the same time (different streams with no event ordering
+ * them, e.g. from two host threads) take work items from each other's queue:
+ * their results are wrong and their waits may end in VT_DEV_TIMEOUT.  Order
+ * such calls (one stream, or events), or use vt_sparse_decode_fused with one
+ * workspace per stream.  After a call that reported VT_DEV_TIMEOUT the
+ * counters may be left nonzero, and later calls on that device may fail the
+ * same way; only a new CUDA context (a new process) starts from zero again.
+ */
+#define VT_STATIC_SCRATCH_BYTES (32u << 20)
+vt_status vt_sparse_decode_fused_static(const vt_paged_kv* kv, const vt_decode_args* a,
+                                        void* out, float* lse, int32_t* sel, int32_t* n_sel,
+                                        void* stream);
+
+/*
  * Workload planner ("a workload planner for balanced GPU scheduling", same
  * article and section): writes to order[0..B) the request indices sorted by
  * page count, longest first (equal counts keep index order), so that long

@@ -23,4 +23,5 @@ from .binding import (  # noqa: F401
     vt_select_pages,
     vt_sparse_decode,
     vt_sparse_decode_fused,
+    vt_sparse_decode_fused_static,
 )

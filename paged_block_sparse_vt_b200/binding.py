@@ -51,7 +51,8 @@ class DecodeArgs(ctypes.Structure):
 
 
 EXPORTS = ("vt_build_centroids", "vt_select_pages", "vt_sparse_decode", "vt_sparse_decode_fused",
-           "vt_fused_workspace_size", "vt_plan_requests", "vt_status_string",
+           "vt_fused_workspace_size", "vt_sparse_decode_fused_static", "vt_plan_requests",
+           "vt_status_string",
            "vt_last_error_detail", "vt_abi_version")
 
 _lock = threading.Lock()
@@ -74,6 +75,7 @@ def load_library(path: str = LIB_PATH):
                 "vt_select_pages": [kv, args, P, P, P],
                 "vt_sparse_decode": [kv, args, P, P, P, P, P],
                 "vt_sparse_decode_fused": [kv, args, P, P, P, P, P, ctypes.c_size_t, P],
+                "vt_sparse_decode_fused_static": [kv, args, P, P, P, P, P],
                 "vt_plan_requests": [P, I32, P, P],
             }
             for name, argtypes in sigs.items():
@@ -248,6 +250,27 @@ def vt_sparse_decode_fused(q, k_pool, v_pool, page_table, seq_lens, centroids, t
                                     _ptr(sel), _ptr(n_sel), _ptr(workspace),
                                     0 if workspace is None else workspace.numel(), _stream(q))
     _check(rc, "vt_sparse_decode_fused")
+    return out, lse, sel, n_sel
+
+
+def vt_sparse_decode_fused_static(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos,
+                                  eos, sm_scale, out=None, lse=None, sel=None, n_sel=None,
+                                  order=None, status=None, head_dim_v=None, want_lse=True):
+    """vt_sparse_decode_fused on the library's own static scratch (no workspace argument).
+
+    Calls on one device share that scratch: they must not overlap on the GPU.
+    """
+    lib = load_library()
+    kv = paged_kv(k_pool, v_pool, head_dim_v)
+    a = decode_args(q, page_table, seq_lens, centroids, topk, bos, eos, sm_scale, order, status)
+    B, hq = q.shape[0], q.shape[1]
+    if out is None:
+        out = torch.empty((B, hq, kv.head_dim_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    rc = lib.vt_sparse_decode_fused_static(ctypes.byref(kv), ctypes.byref(a), out.data_ptr(),
+                                           _ptr(lse), _ptr(sel), _ptr(n_sel), _stream(q))
+    _check(rc, "vt_sparse_decode_fused_static")
     return out, lse, sel, n_sel
 
 

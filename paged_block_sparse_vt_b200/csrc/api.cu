@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
+#include <mutex>
 
 #include "decode_params.cuh"
 
@@ -17,11 +18,11 @@ cudaError_t launch_mla_decode(const DecodeParams& p, int mode, int G, int C, cud
 int mla_smem_bytes(int G, int cand_cap, int key_cap, int kmax, int pages_per_cta);
 int mla_max_pages_per_cta();
 cudaError_t launch_plan(const int32_t* seq_lens, int B, int32_t* order, cudaStream_t s);
-size_t persist_workspace_bytes(const DecodeParams& p, int G, int Dv);
+size_t persist_workspace_bytes(const DecodeParams& p, int G, int Dv, int64_t unit_cap);
 int persist_smem_bytes(const DecodeParams& p, int D, int G);
 int persist_max_batch();
-cudaError_t launch_persist_fused(const DecodeParams& p, int D, int G, void* ws, int sm_count,
-                                 cudaStream_t s);
+cudaError_t launch_persist_fused(const DecodeParams& p, int D, int G, void* ws, int64_t unit_cap,
+                                 int sm_count, cudaStream_t s);
 }  // namespace vt
 
 using namespace vt;
@@ -194,9 +195,10 @@ bool use_persistent(const Shape& sh, const vt_decode_args* a) {
   return sh.path == kPathGqa && a->batch >= 1 && a->batch <= persist_max_batch();
 }
 
+// unit_cap: units the persistent path's counter arrays are laid out for (0: exactly B * Hkv)
 vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int mode,
                             int32_t* sel, int32_t* n_sel, void* out, float* lse, void* ws,
-                            size_t ws_bytes, void* stream) {
+                            size_t ws_bytes, void* stream, int64_t unit_cap = 0) {
   Shape sh;
   DecodeParams p;
   vt_status s = fill_params(kv, a, mode != kDecode, &sh, &p);
@@ -213,7 +215,7 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
   p.lse = lse;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (mode == kFused && use_persistent(sh, a)) {
-    const size_t need = persist_workspace_bytes(p, sh.G, sh.Dv);
+    const size_t need = persist_workspace_bytes(p, sh.G, sh.Dv, unit_cap);
     if (!ws || ws_bytes < need)
       return fail(VT_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need,
                   ws ? ws_bytes : (size_t)0);
@@ -221,7 +223,7 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
       return fail(VT_ERR_INVALID_ARG, "workspace not 256-byte aligned");
     const int bytes = persist_smem_bytes(p, sh.D, sh.G);
     if (bytes > 227 * 1024) return fail(VT_ERR_UNSUPPORTED, "shared memory need %d B too large", bytes);
-    cudaError_t e = launch_persist_fused(p, sh.D, sh.G, ws, sm_count(), st);
+    cudaError_t e = launch_persist_fused(p, sh.D, sh.G, ws, unit_cap, sm_count(), st);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return ok();
   }
@@ -245,6 +247,35 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
   }
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return ok();
+}
+
+// ---- the library-owned scratch of vt_sparse_decode_fused_static ----------------------------
+
+// One per device the module is loaded on, zero-filled by CUDA at load.  The persistent
+// kernel leaves its counters at zero after every complete call, so it is never cleared here.
+static __device__ __align__(256) unsigned char g_static_scratch[VT_STATIC_SCRATCH_BYTES];
+// Its per-unit counters are laid out for this many units whatever the call's shape, so they
+// sit at the same offsets in every call and never overlap another call's data.
+constexpr int64_t kStaticUnitCap = 65536;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices];  // device address of g_static_scratch, looked up once per device
+
+cudaError_t static_scratch_address(void** addr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return e;
+    g_static_addr[dev] = p;
+  }
+  *addr = g_static_addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -291,7 +322,41 @@ size_t vt_fused_workspace_size(const vt_paged_kv* kv, const vt_decode_args* a) {
   DecodeParams p;
   if (fill_params(kv, a, true, &sh, &p) != VT_OK) return 0;
   if (!use_persistent(sh, a)) return 0;
-  return persist_workspace_bytes(p, sh.G, sh.Dv);
+  return persist_workspace_bytes(p, sh.G, sh.Dv, 0);
+}
+
+vt_status vt_sparse_decode_fused_static(const vt_paged_kv* kv, const vt_decode_args* a,
+                                        void* out, float* lse, int32_t* sel, int32_t* n_sel,
+                                        void* stream) {
+  // 0 for arguments the fused call rejects (it then reports why) and for shapes that need
+  // no workspace
+  size_t need = 0;
+  {
+    Shape sh;
+    DecodeParams p;
+    if (fill_params(kv, a, true, &sh, &p) == VT_OK && use_persistent(sh, a)) {
+      if ((int64_t)a->batch * kv->num_kv_heads > kStaticUnitCap)
+        return fail(VT_ERR_UNSUPPORTED, "B * Hkv > %lld units for the static scratch",
+                    (long long)kStaticUnitCap);
+      need = persist_workspace_bytes(p, sh.G, sh.Dv, kStaticUnitCap);
+    }
+  }
+  if (need > (size_t)VT_STATIC_SCRATCH_BYTES)
+    return fail(VT_ERR_UNSUPPORTED, "needs %zu bytes of scratch; the static scratch holds %zu",
+                need, (size_t)VT_STATIC_SCRATCH_BYTES);
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  if (need > 0) {
+    // the call-level checks of the fused call, before any CUDA call
+    if (!out) return fail(VT_ERR_INVALID_ARG, "out is NULL");
+    if ((sel == nullptr) != (n_sel == nullptr))
+      return fail(VT_ERR_INVALID_ARG, "sel and n_sel must both be given or both be NULL");
+    cudaError_t e = static_scratch_address(&ws);
+    if (e != cudaSuccess) return cuda_fail(e, "static scratch address");
+    ws_bytes = VT_STATIC_SCRATCH_BYTES;
+  }
+  return launch_query_side(kv, a, kFused, sel, n_sel, out, lse, ws, ws_bytes, stream,
+                           kStaticUnitCap);
 }
 
 vt_status vt_plan_requests(const int32_t* seq_lens, int32_t batch, int32_t* order, void* stream) {

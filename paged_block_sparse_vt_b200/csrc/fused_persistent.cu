@@ -94,15 +94,19 @@ struct PersistWsLayout {
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-static PersistWsLayout persist_ws_layout(const DecodeParams& p, int G, int Dv) {
+// unit_cap >= B * Hkv: units the counter arrays are laid out for.  The counters are the only
+// part that must be zero before a call; with a fixed unit_cap they sit at the same offsets for
+// every shape, so calls of different shapes can share one buffer.
+static PersistWsLayout persist_ws_layout(const DecodeParams& p, int G, int Dv, int64_t unit_cap) {
   const PersistGeom g = persist_geom(p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
   const size_t U = (size_t)p.B * p.Hkv;
+  const size_t cap = unit_cap > (int64_t)U ? (size_t)unit_cap : U;
   const size_t cand = U * g.nch_max * g.kc;
   PersistWsLayout L;
   size_t o = 0;
   L.ctr = o;       o += align256(2 * sizeof(int32_t));
-  L.unit_done = o; o += align256(U * sizeof(int32_t));
-  L.att_cnt = o;   o += align256(U * sizeof(int32_t));
+  L.unit_done = o; o += align256(cap * sizeof(int32_t));
+  L.att_cnt = o;   o += align256(cap * sizeof(int32_t));
   L.ckey = o;      o += align256(cand * sizeof(uint32_t));
   L.coff = o;      o += align256(cand * sizeof(uint16_t));
   L.part = o;      o += align256(U * g.A * G * (Dv + 2) * sizeof(float));
@@ -521,8 +525,8 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
 
 // ---- host side ----------------------------------------------------------------------------
 
-size_t persist_workspace_bytes(const DecodeParams& p, int G, int Dv) {
-  return persist_ws_layout(p, G, Dv).total;
+size_t persist_workspace_bytes(const DecodeParams& p, int G, int Dv, int64_t unit_cap) {
+  return persist_ws_layout(p, G, Dv, unit_cap).total;
 }
 
 int persist_smem_bytes(const DecodeParams& p, int D, int G) {
@@ -564,11 +568,11 @@ static cudaError_t dispatch_persist_g(const DecodeParams& p, const PersistWs& w,
   }
 }
 
-// Launch the persistent kernel on `ws` (persist_workspace_bytes() bytes, zero-filled once
-// before first use): as many CTAs as fit on the sm_count SMs at once.
-cudaError_t launch_persist_fused(const DecodeParams& p, int D, int G, void* ws, int sm_count,
-                                 cudaStream_t s) {
-  const PersistWsLayout L = persist_ws_layout(p, G, D);
+// Launch the persistent kernel on `ws` (persist_workspace_bytes() bytes for the same
+// unit_cap, counters zero): as many CTAs as fit on the sm_count SMs at once.
+cudaError_t launch_persist_fused(const DecodeParams& p, int D, int G, void* ws, int64_t unit_cap,
+                                 int sm_count, cudaStream_t s) {
+  const PersistWsLayout L = persist_ws_layout(p, G, D, unit_cap);
   unsigned char* base = static_cast<unsigned char*>(ws);
   PersistWs w;
   w.ctr = reinterpret_cast<int32_t*>(base + L.ctr);
