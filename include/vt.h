@@ -166,10 +166,11 @@ vt_status vt_sparse_decode(const vt_paged_kv* kv, const vt_decode_args* a, const
  * derive from seq_lens themselves (a->order is not used there), which keeps
  * every SM busy on batches of very uneven lengths; it needs `workspace`: device memory of vt_fused_workspace_size()
  * bytes, 256-byte aligned, ZERO-FILLED ONCE when allocated.  Every call
- * leaves it ready for the next one, so it is zeroed only once, but calls that
- * share a workspace must not overlap on the GPU (use one stream, or one
- * workspace per stream); after a call that reported VT_DEV_TIMEOUT, zero it
- * again.  When vt_fused_workspace_size() is 0 (MLA, or B > 2048) no
+ * leaves it ready for the next one with the same B * Hkv, so it is zeroed
+ * only once (its counter arrays are laid out for B * Hkv units: zero it again
+ * before a call with another B * Hkv).  Calls that share a workspace must not
+ * overlap on the GPU (use one stream, or one workspace per stream); after a
+ * call that reported VT_DEV_TIMEOUT, zero it again.  When vt_fused_workspace_size() is 0 (MLA, or B > 2048) no
  * workspace is used and `workspace` may be NULL.
  */
 vt_status vt_sparse_decode_fused(const vt_paged_kv* kv, const vt_decode_args* a, void* out,

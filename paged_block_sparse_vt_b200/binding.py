@@ -218,8 +218,9 @@ def fused_workspace(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bo
                     head_dim_v=None) -> Optional[torch.Tensor]:
     """A zero-filled workspace for vt_sparse_decode_fused (None when none is needed).
 
-    Zero it once; every call leaves it ready for the next.  Calls sharing one workspace must
-    not overlap on the GPU.
+    Zero it once; every call leaves it ready for the next call with the same B * Hkv (zero it
+    again before one with another B * Hkv).  Calls sharing one workspace must not overlap on
+    the GPU.
     """
     n = vt_fused_workspace_size(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos,
                                 eos, head_dim_v)
