@@ -10,8 +10,9 @@
 // and kernel fusion); the thread on digg.com, closing reply (batch heterogeneity is where
 // sparse-attention speedups are lost).
 //
-// Work items, claimed in order through one global counter (each CTA claims its next item
-// before it starts on the current one, so the counter's latency is hidden):
+// Work items, claimed in order through one global counter (a CTA claims its next item when
+// the streaming part of the current one is done, so the counter's latency is hidden by the
+// current item's tail and the queue order still follows the CTAs' actual progress):
 //   scan items   -- (request, KV head, chunk of kChunk candidate pages), in request order,
 //                   each unit's chunks consecutive.  Every warp streams its rows of the
 //                   chunk's fp32 centroids through a cp.async ring and dots them with the
@@ -20,7 +21,7 @@
 //                   score key and offset, ascending by page) before counting the chunk done.
 //                   The union of the chunks' top-k holds the unit's top-k: a key outside its
 //                   chunk's top-k has k keys above it in that chunk alone;
-//   attention    -- (unit, piece of kPiecePages selected pages), after every scan item.  The
+//   attention    -- (unit, piece of at most kPiecePages selected pages), after every scan item.  The
 //   items           CTA waits until all of the unit's chunks are counted (every chunk was
 //                   claimed before this item and scan items never wait, so the wait ends),
 //                   merges the candidates with the same exact top-k, attends the pages of its
@@ -28,8 +29,10 @@
 //                   stores a partial (max, sum, acc); the CTA that completes a unit's last
 //                   piece merges the partials and writes the bf16 output and the lse.
 // The schedule (scan items per request and their prefix) is computed by every CTA from the
-// sequence lengths at start, so the call is one launch.  Every counter is reset by the CTA
-// that last uses it, so the workspace needs zero-filling only once.
+// sequence lengths at start, so the call is one launch.  The per-unit counters are reset by
+// the CTA that last uses them and the claim counter runs on across launches (each launch
+// numbers its items from where the previous one stopped), so the workspace needs
+// zero-filling only once and no CTA waits for the others on its way out.
 #include "decode_params.cuh"
 #include "gqa_attend.cuh"
 #include "topk.cuh"
@@ -40,8 +43,9 @@ constexpr int kPersistThreads = 128;
 constexpr int kPersistWarps = kPersistThreads / 32;
 constexpr int kChunk = 256;      // candidate pages per scan item (64 per warp)
 constexpr int kScanRing = 4;     // 8-row centroid batches per warp ring (3 landing)
-constexpr int kPiecePages = 16;  // selected pages per attention item (4 per warp)
+constexpr int kPiecePages = 16;  // most selected pages per attention item (4 per warp)
 constexpr int kMaxPlanB = 2048;  // requests the persistent path takes (schedule kept in smem)
+constexpr int kPersistMinCtas = 3;  // CTAs per SM the registers must allow (<= 168 per thread)
 
 // ---- sizes derived from the call ----------------------------------------------------------
 
@@ -50,6 +54,7 @@ struct PersistGeom {
   int nch_max;   // chunks of such a row
   int kc;        // candidates a chunk keeps: min(topk, kChunk)
   int A;         // attention pieces per unit
+  int pp;        // selected pages per piece: kmax split evenly, at most kPiecePages
   int cmax;      // candidates one unit merges at most
 };
 
@@ -61,6 +66,7 @@ __host__ __device__ inline PersistGeom persist_geom(int64_t pt_stride, int topk,
   g.nch_max = (g.max_cand + kChunk - 1) / kChunk;
   g.kc = topk < kChunk ? (topk > 0 ? topk : 1) : kChunk;
   g.A = (kmax + kPiecePages - 1) / kPiecePages;
+  g.pp = (kmax + g.A - 1) / g.A;
   const int64_t c = (int64_t)g.nch_max * g.kc;
   g.cmax = c < g.max_cand ? (int)c : g.max_cand;
   return g;
@@ -78,18 +84,19 @@ __host__ __device__ inline int chunks_of(int L, int64_t pt_stride, int topk, int
 // ---- workspace ----------------------------------------------------------------------------
 
 struct PersistWs {
-  int32_t* ctr;        // [2]: items claimed, CTAs finished
+  uint32_t* ctr;       // [2]: claims ever made (mod 2^32), the claim count when this launch began
   int32_t* unit_done;  // [U]: chunks of the unit whose candidates are stored
   int32_t* att_cnt;    // [U]: attention pieces of the unit done
   uint32_t* ckey;      // [U][nch_max][kc]: ordered score keys of each chunk's top-k
   uint16_t* coff;      // [U][nch_max][kc]: their offsets in the chunk, ascending
+  int32_t* cpid;       // [U][nch_max][kc]: their page ids (-1 where the id was out of range)
   float* part;         // [U][A][G][Dv+2]: attention partials
   PersistGeom g;
   int units;
 };
 
 struct PersistWsLayout {
-  size_t ctr, unit_done, att_cnt, ckey, coff, part, total;
+  size_t ctr, unit_done, att_cnt, ckey, coff, cpid, part, total;
 };
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -104,11 +111,12 @@ static PersistWsLayout persist_ws_layout(const DecodeParams& p, int G, int Dv, i
   const size_t cand = U * g.nch_max * g.kc;
   PersistWsLayout L;
   size_t o = 0;
-  L.ctr = o;       o += align256(2 * sizeof(int32_t));
+  L.ctr = o;       o += align256(2 * sizeof(uint32_t));
   L.unit_done = o; o += align256(cap * sizeof(int32_t));
   L.att_cnt = o;   o += align256(cap * sizeof(int32_t));
   L.ckey = o;      o += align256(cand * sizeof(uint32_t));
   L.coff = o;      o += align256(cand * sizeof(uint16_t));
+  L.cpid = o;      o += align256(cand * sizeof(int32_t));
   L.part = o;      o += align256(U * g.A * G * (Dv + 2) * sizeof(float));
   L.total = o;
   return L;
@@ -137,7 +145,7 @@ struct PersistShape : PageTile<D> {
 };
 
 struct PersistSmem {
-  int prefix, keys, sel, phys, misc, region, total;
+  int prefix, keys, pids, sel, phys, misc, region, total;
 };
 
 __host__ __device__ inline PersistSmem persist_smem_layout(int D, int G, int B,
@@ -146,6 +154,7 @@ __host__ __device__ inline PersistSmem persist_smem_layout(int D, int G, int B,
   int o = 0;
   s.prefix = o; o += align16((B + 1) * 4);
   s.keys = o;   o += align16(kChunk * 4);
+  s.pids = o;   o += align16(kChunk * 4);
   s.sel = o;    o += align16(kPiecePages * 4);
   s.phys = o;   o += align16(kPiecePages * 4);
   s.misc = o;   o += align16(64 * 4);
@@ -153,7 +162,11 @@ __host__ __device__ inline PersistSmem persist_smem_layout(int D, int G, int B,
   s.region = o;  // one of: scan rings | top-k scratch | page rings | attention partials
   const int scan = kPersistWarps * kScanRing * 8 * D * 4;
   const int att = kPersistWarps * 2 * 2 * kPage * (D + 8) * 2;
-  const int merge = align16(g.cmax * 4) + align16(g.cmax * 2) + align16((kTopkBins + 64) * 4);
+  // merge of up to 2 NT candidates: keys, logical and physical pages, small_topk scratch;
+  // of more: keys, offsets, block_topk scratch
+  const int merge_small = 3 * 2 * kPersistThreads * 4 + SmallTopk<kPersistThreads>::BYTES;
+  const int merge_big = align16(g.cmax * 4) + align16(g.cmax * 2) + align16((kTopkBins + 64) * 4);
+  const int merge = merge_small > merge_big ? merge_small : merge_big;
   const int comb = align16(kPersistWarps * G * (D + 2) * 4) + align16(G * (D + 2) * 4) +
                    align16(g.A * G * (D + 2) * 4);
   int r = scan;
@@ -165,7 +178,7 @@ __host__ __device__ inline PersistSmem persist_smem_layout(int D, int G, int B,
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const DecodeParams p,
+__global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fused_kernel(const DecodeParams p,
                                                                         const PersistWs w) {
   using S = PersistShape<D>;
   constexpr int NT = kPersistThreads;
@@ -174,6 +187,8 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
   constexpr int RPS = 32 / LPR_S;  // centroid rows per warp step
   constexpr int SN = 8 / RPS;      // values per lane per batch of 8 rows
   static_assert(D == 64 || D == 128, "GQA path covers head_dim 64 and 128");
+  static_assert(SmallTopk<kPersistThreads>::BYTES <= kScanRing * 8 * D * 4,
+                "the chunk top-k scratch fits in warp 0's scan ring");
 
   extern __shared__ __align__(128) unsigned char smem[];
   const PersistGeom gm = w.g;
@@ -181,6 +196,7 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
   const PersistSmem Ls = persist_smem_layout(D, G, p.B, gm);
   int* s_prefix = reinterpret_cast<int*>(smem + Ls.prefix);
   uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem + Ls.keys);
+  int* s_pids = reinterpret_cast<int*>(smem + Ls.pids);  // page ids of the chunk's rows
   int* s_sel = reinterpret_cast<int*>(smem + Ls.sel);
   int* s_phys = reinterpret_cast<int*>(smem + Ls.phys);
   int* s_misc = reinterpret_cast<int*>(smem + Ls.misc);  // [0] item, [1] flag, [8..] scan
@@ -189,8 +205,25 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+  // Launched as a programmatic dependent of the previous kernel on the stream: the CTAs may
+  // be placed while that kernel still runs, and nothing in global memory is touched before it
+  // has completed.  The next such launch may likewise be placed early.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+
+  uint32_t qbase = 0;  // thread 0: the claim count when this launch began
+  auto claim = [&]() { return (int)(atomicAdd(w.ctr + 0, 1u) - qbase); };
+
   // ---- schedule: exclusive prefix of scan items over the requests, in request order
   {
+    // the first item, claimed now so that the claim overlaps the prefix.  Items are numbered
+    // from the claim count at which this launch began (qbase), so the counter is never reset:
+    // the launch's last claim stores the next launch's qbase.
+    int first = 0;
+    if (tid == 0) {
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(qbase) : "l"(w.ctr + 1) : "memory");
+      first = claim();
+    }
     const int per = (p.B + NT - 1) / NT;
     const int i0 = min(p.B, tid * per), i1 = min(p.B, i0 + per);
     int run = 0;
@@ -215,19 +248,28 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
       acc += c;
     }
     if (tid == NT - 1) s_prefix[p.B] = base + x;
-    if (tid == 0) s_misc[0] = atomicAdd(w.ctr + 0, 1);
+    if (tid == 0) s_misc[0] = first;
     __syncthreads();
   }
   const int scan_items = s_prefix[p.B];
   const int total_items = scan_items + w.units * A;
 
+  // A counter that thread 0 bumps (release) once the CTA has passed the barrier at the end
+  // of the item that produced the counted data, so that the fence overlaps the next item.
+  int32_t* pending = nullptr;
   for (;;) {
     const int t = s_misc[0];
     __syncthreads();  // every thread has read the item before the next claim is stored
-    if (t >= total_items) break;
-    // claim the next item now; its number is only stored (and waited for) at the end
-    int next = 0;
-    if (tid == 0) next = atomicAdd(w.ctr + 0, 1);
+    if (t >= total_items) {
+      // Every CTA makes one claim per item plus one that ends it, so the launch's claims are
+      // numbered 0 .. total_items + gridDim.x - 1.  The CTA holding the last one knows that
+      // every CTA has read qbase, and sets it for the next launch.
+      if (tid == 0 && t == total_items + (int)gridDim.x - 1)
+        w.ctr[1] = qbase + (uint32_t)total_items + gridDim.x;
+      break;
+    }
+    // the next item, claimed by thread 0 once this item's streaming is done (or at its end)
+    int next = -1;
 
     if (t < scan_items) {
       // ---------------------------------------------------------------- scan item
@@ -274,6 +316,8 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
         if (pidA < 0 || pidA >= p.num_pages) pidA = -1;
         if (pidB < 0 || pidB >= p.num_pages) pidB = -1;
       }
+      if (lane < myrows) s_pids[warp + NW * lane] = pidA;
+      if (lane + 32 < myrows) s_pids[warp + NW * (lane + 32)] = pidB;
       const uint32_t ring = region_u32 + warp * kScanRing * 8 * S::C_ROW;
       const float* cbase = p.centroids + (int64_t)h * D;
       const int64_t cstride = (int64_t)p.Hkv * D;
@@ -294,6 +338,7 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
         }
         cp_async_commit();
       };
+      uint32_t klo = 0xffffffffu, khi = 0u;  // range of the keys this lane stores
 #pragma unroll
       for (int bt = 0; bt < kScanRing - 1; ++bt) issue(bt);
       for (int bt = 0; bt < batches; ++bt) {
@@ -317,25 +362,47 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
         exchange_reduce<SN, LPR_S>(v, lane);
         const int i = bt * 8 + exchange_index<SN, LPR_S>(lane) * RPS + sub;
         const int pg = page_of_lane(pidA, pidB, i);
-        if ((ch % (LPR_S / SN)) == 0 && i < myrows)
-          s_keys[warp + NW * i] = score_key(pg >= 0 ? v[0] : -INFINITY);
+        if ((ch % (LPR_S / SN)) == 0 && i < myrows) {
+          const uint32_t key = score_key(pg >= 0 ? v[0] : -INFINITY);
+          s_keys[warp + NW * i] = key;
+          klo = min(klo, key);
+          khi = max(khi, key);
+        }
         __syncwarp();  // every lane is done with the slot before it is refilled
       }
       cp_async_wait<0>();
+      if (tid == 0) next = claim();
+      klo = __reduce_min_sync(kFull, klo);
+      khi = __reduce_max_sync(kFull, khi);
+      if (lane == 0) {
+        s_misc[16 + warp] = (int)klo;
+        s_misc[16 + NW + warp] = (int)khi;
+      }
+      // the top-k scratch lies in warp 0's ring, which only warp 0 has used
+      unsigned char* tk = region;
+      if (warp == 0)
+        for (int i = lane; i < SmallTopk<NT>::HIST / 4; i += 32)
+          reinterpret_cast<int4*>(tk)[i] = make_int4(0, 0, 0, 0);
       __syncthreads();  // all scores of the chunk are in s_keys; the rings are free
+      klo = 0xffffffffu;
+      khi = 0u;
+#pragma unroll
+      for (int k = 0; k < NW; ++k) {
+        klo = min(klo, (uint32_t)s_misc[16 + k]);
+        khi = max(khi, (uint32_t)s_misc[16 + NW + k]);
+      }
       // exact top-kc of the chunk, stored in ascending page order
       const int kc = min(gm.kc, cnt);
       const int64_t cb = ((int64_t)u * gm.nch_max + c) * gm.kc;
       uint32_t* ck = w.ckey + cb;
       uint16_t* co = w.coff + cb;
-      int* hist = reinterpret_cast<int*>(region);
-      block_topk<NT>(s_keys, cnt, kc, hist, hist + kTopkBins, [&](int j, int pos) {
+      int32_t* cp = w.cpid + cb;
+      small_topk<NT>(s_keys, cnt, kc, klo, khi, tk, [&](int j, int pos) {
         ck[pos] = s_keys[j];
         co[pos] = (uint16_t)j;
+        cp[pos] = s_pids[j];
       });
-      __threadfence();  // this thread's candidates before the unit counter moves
-      __syncthreads();
-      if (tid == 0) atomicAdd(w.unit_done + u, 1);
+      pending = w.unit_done + u;  // counted after the item's closing barrier
     } else {
       // ---------------------------------------------------------------- attention item
       const int a = t - scan_items;
@@ -347,8 +414,8 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
       const bool dense = n <= p.kmax;
       const int nch = chunks_of(L, p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
       const int ns = !valid ? 0 : (dense ? n : p.kmax);
-      const int j0 = piece * kPiecePages;
-      const int np = max(0, min(ns - j0, kPiecePages));
+      const int j0 = piece * gm.pp;
+      const int np = max(0, min(ns - j0, gm.pp));
       const bool write_sel = piece == 0 && p.sel != nullptr;
       int32_t* selrow = write_sel ? p.sel + (int64_t)u * p.kmax : nullptr;
       if (tid == 0 && piece == 0) {
@@ -377,38 +444,97 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
         ok = s_misc[1];
       }
       if (ok) {
-        // ---- the logical pages of this piece into s_sel[0, np)
+        // ---- the logical pages of this piece into s_sel[0, np), their page ids into s_phys
+        const int32_t* ptrow = p.page_table + (int64_t)b * p.pt_stride;
+        auto phys_of = [&](int lp) {
+          int pg = ptrow[lp];
+          if (pg < 0 || pg >= p.num_pages) {
+            flag(p.status, VT_DEV_BAD_PAGE);
+            pg = -1;
+          }
+          return pg;
+        };
+        bool have_phys = false;
         if (nch > 0) {
           const int m = n - p.bos - p.eos;
           const int kc = gm.kc;
           const int C = (nch - 1) * kc + min(kc, m - (nch - 1) * kChunk);
-          uint32_t* keys = reinterpret_cast<uint32_t*>(region);
-          uint16_t* offs = reinterpret_cast<uint16_t*>(region + align16(gm.cmax * 4));
-          int* hist = reinterpret_cast<int*>(region + align16(gm.cmax * 4) + align16(gm.cmax * 2));
           const int64_t cb = (int64_t)u * gm.nch_max * kc;  // chunks are contiguous
-          for (int j = tid; j < C; j += NT) {
-            keys[j] = __ldcg(w.ckey + cb + j);
-            offs[j] = __ldcg(w.coff + cb + j);
-          }
           const int bos = p.bos, topk = p.topk;
           for (int q = tid; q < np; q += NT) {  // reserved pages of the piece
             const int pos = j0 + q;
-            if (pos < bos) s_sel[q] = pos;
-            else if (pos >= bos + topk) s_sel[q] = n - p.eos + (pos - bos - topk);
+            if (pos < bos || pos >= bos + topk) {
+              const int lp = pos < bos ? pos : n - p.eos + (pos - bos - topk);
+              s_sel[q] = lp;
+              s_phys[q] = phys_of(lp);
+            }
           }
           if (write_sel) {
             for (int j = tid; j < bos; j += NT) selrow[j] = j;
             for (int j = tid; j < p.eos; j += NT) selrow[bos + topk + j] = n - p.eos + j;
           }
-          __syncthreads();
-          // candidate j of chunk j / kc sits at offset offs[j] of it; candidates are in
-          // ascending page order, so block_topk's ties (lowest position) go to the lowest page
-          block_topk<NT>(keys, C, topk, hist, hist + kTopkBins, [&](int j, int pos) {
-            const int lp = bos + (j / kc) * kChunk + offs[j];
-            const int q = bos + pos - j0;
-            if (q >= 0 && q < kPiecePages) s_sel[q] = lp;
-            if (write_sel) selrow[bos + pos] = lp;
-          });
+          // candidate j of chunk j / kc sits at offset coff[j] of it; candidates are in
+          // ascending page order, so ties (lowest position) go to the lowest page
+          if (C <= 2 * NT) {
+            // keys, logical pages and page ids of the candidates, fetched together
+            uint32_t* keys = reinterpret_cast<uint32_t*>(region);
+            int* lps = reinterpret_cast<int*>(region + 2 * NT * 4);
+            int* pids = reinterpret_cast<int*>(region + 4 * NT * 4);
+            unsigned char* tk = region + 6 * NT * 4;
+            for (int i = tid; i < SmallTopk<NT>::HIST / 4; i += NT)
+              reinterpret_cast<int4*>(tk)[i] = make_int4(0, 0, 0, 0);
+            uint32_t klo = 0xffffffffu, khi = 0u;
+            for (int j = tid; j < C; j += NT) {
+              const uint32_t key = __ldcg(w.ckey + cb + j);
+              const int lp = bos + (j / kc) * kChunk + __ldcg(w.coff + cb + j);
+              keys[j] = key;
+              lps[j] = lp;
+              pids[j] = __ldcg(w.cpid + cb + j);
+              klo = min(klo, key);
+              khi = max(khi, key);
+            }
+            klo = __reduce_min_sync(kFull, klo);
+            khi = __reduce_max_sync(kFull, khi);
+            if (lane == 0) {
+              s_misc[16 + warp] = (int)klo;
+              s_misc[16 + NW + warp] = (int)khi;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int k = 0; k < NW; ++k) {
+              klo = min(klo, (uint32_t)s_misc[16 + k]);
+              khi = max(khi, (uint32_t)s_misc[16 + NW + k]);
+            }
+            small_topk<NT>(keys, C, topk, klo, khi, tk, [&](int j, int pos) {
+              const int q = bos + pos - j0;
+              if (q >= 0 && q < np) {
+                s_sel[q] = lps[j];
+                int pg = pids[j];
+                if (pg < 0 || pg >= p.num_pages) {
+                  flag(p.status, VT_DEV_BAD_PAGE);
+                  pg = -1;
+                }
+                s_phys[q] = pg;
+              }
+              if (write_sel) selrow[bos + pos] = lps[j];
+            });
+            have_phys = true;
+          } else {
+            uint32_t* keys = reinterpret_cast<uint32_t*>(region);
+            uint16_t* offs = reinterpret_cast<uint16_t*>(region + align16(gm.cmax * 4));
+            int* hist = reinterpret_cast<int*>(region + align16(gm.cmax * 4) + align16(gm.cmax * 2));
+            for (int j = tid; j < C; j += NT) {
+              keys[j] = __ldcg(w.ckey + cb + j);
+              offs[j] = __ldcg(w.coff + cb + j);
+            }
+            __syncthreads();
+            block_topk<NT>(keys, C, topk, hist, hist + kTopkBins, [&](int j, int pos) {
+              const int lp = bos + (j / kc) * kChunk + offs[j];
+              const int q = bos + pos - j0;
+              if (q >= 0 && q < np) s_sel[q] = lp;
+              if (write_sel) selrow[bos + pos] = lp;
+            });
+          }
         } else {
           // dense (every page, in order) or, with topk == 0, the reserved pages alone
           const bool resv = valid && !dense;
@@ -420,16 +546,10 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
             for (int j = tid; j < p.kmax; j += NT) selrow[j] = j < ns ? page_at(j) : -1;
         }
         __syncthreads();
-        const int32_t* ptrow = p.page_table + (int64_t)b * p.pt_stride;
-        if (tid < np) {
-          int pg = ptrow[s_sel[tid]];
-          if (pg < 0 || pg >= p.num_pages) {
-            flag(p.status, VT_DEV_BAD_PAGE);
-            pg = -1;
-          }
-          s_phys[tid] = pg;
+        if (!have_phys) {
+          if (tid < np) s_phys[tid] = phys_of(s_sel[tid]);
+          __syncthreads();
         }
-        __syncthreads();
         // ---- warp w: pages w + NW i (i < 4) of the piece through a two-slot ring
         const int last_valid = L - kPage * (n - 1);
         const uint32_t ring = region_u32 + warp * 2 * S::SLOT;
@@ -459,6 +579,7 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
           __syncwarp();
         }
         cp_async_wait<0>();
+        if (tid == 0) next = claim();
         __syncthreads();  // every warp is done with the staged tiles: partials may reuse them
         float* s_wp = reinterpret_cast<float*>(region);  // [NW][G][D+2]
         float* s_cp = s_wp + NW * G * (D + 2);            // [G][D+2]
@@ -469,28 +590,45 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
         __syncthreads();
         int fin = 1;
         if (A > 1) {
-          float* dst = w.part + ((int64_t)u * A + piece) * G * (D + 2);
-          for (int i = tid; i < G * (D + 2); i += NT) dst[i] = s_cp[i];
-          __threadfence();
-          __syncthreads();
-          if (tid == 0) {
-            const int done = atomicAdd(w.att_cnt + u, 1);
-            const int last = (done == A - 1);
-            if (last) {  // every piece of u has waited and stored: reset u's counters
-              w.att_cnt[u] = 0;
-              w.unit_done[u] = 0;
-              __threadfence();
+          if (piece < A - 1) {
+            // publish this piece's partial and move on: the unit's last piece merges them
+            float* dst = w.part + ((int64_t)u * A + piece) * G * (D + 2);
+            for (int i = tid; i < G * (D + 2); i += NT) dst[i] = s_cp[i];
+            pending = w.att_cnt + u;
+            fin = 0;
+          } else {
+            // the last piece waits for the other A - 1 partials; their items were claimed
+            // before this one and never wait on a later item, so the wait ends
+            if (tid == 0) {
+              int okm = 1;
+              if (ld_acquire(w.att_cnt + u) < A - 1) {
+                const unsigned long long t0 = global_ns();
+                for (;;) {
+                  __nanosleep(64);
+                  if (ld_acquire(w.att_cnt + u) >= A - 1) break;
+                  if (global_ns() - t0 > kWaitNs) {
+                    flag(p.status, kDevTimeout);
+                    okm = 0;
+                    break;
+                  }
+                }
+              }
+              s_misc[1] = okm;
             }
-            s_misc[1] = last;
-          }
-          __syncthreads();
-          fin = s_misc[1];
-          if (fin) {
-            const float* src = w.part + (int64_t)u * A * G * (D + 2);
-            for (int i = tid; i < A * G * (D + 2); i += NT) s_all[i] = __ldcg(src + i);
             __syncthreads();
-            merge_partials<G, D>(s_all, A, s_cp, tid, NT);
-            __syncthreads();
+            fin = s_misc[1];
+            if (fin) {
+              const float* src = w.part + (int64_t)u * A * G * (D + 2);
+              for (int i = tid; i < (A - 1) * G * (D + 2); i += NT) s_all[i] = __ldcg(src + i);
+              for (int i = tid; i < G * (D + 2); i += NT) s_all[(A - 1) * G * (D + 2) + i] = s_cp[i];
+              __syncthreads();
+              merge_partials<G, D>(s_all, A, s_cp, tid, NT);
+              __syncthreads();
+              if (tid == 0) {  // every piece of u is past its waits: reset u's counters
+                w.att_cnt[u] = 0;
+                w.unit_done[u] = 0;
+              }
+            }
           }
         } else if (tid == 0 && nch > 0) {
           w.unit_done[u] = 0;
@@ -507,20 +645,16 @@ __global__ void __launch_bounds__(kPersistThreads) persist_fused_kernel(const De
         }
       }
     }
-    if (tid == 0) s_misc[0] = next;
+    if (tid == 0) s_misc[0] = next >= 0 ? next : claim();
     __syncthreads();
-  }
-
-  // leave: the last CTA out resets the queue for the next launch
-  if (tid == 0) {
-    __threadfence();
-    const int out = atomicAdd(w.ctr + 1, 1);
-    if (out == (int)gridDim.x - 1) {
-      w.ctr[0] = 0;
+    if (tid == 0 && pending != nullptr) {
+      // the barrier above ordered every thread's stores of the item before this fence
       __threadfence();
-      w.ctr[1] = 0;
+      atomicAdd(pending, 1);
+      pending = nullptr;
     }
   }
+
 }
 
 // ---- host side ----------------------------------------------------------------------------
@@ -548,8 +682,17 @@ static cudaError_t launch_persist_t(const DecodeParams& p, const PersistWs& w, i
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kPersistThreads, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  kern<<<sm_count * per_sm, kPersistThreads, smem, stream>>>(p, w);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sm_count * per_sm);
+  cfg.blockDim = dim3(kPersistThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p, w);
 }
 
 template <int D>
@@ -575,11 +718,12 @@ cudaError_t launch_persist_fused(const DecodeParams& p, int D, int G, void* ws, 
   const PersistWsLayout L = persist_ws_layout(p, G, D, unit_cap);
   unsigned char* base = static_cast<unsigned char*>(ws);
   PersistWs w;
-  w.ctr = reinterpret_cast<int32_t*>(base + L.ctr);
+  w.ctr = reinterpret_cast<uint32_t*>(base + L.ctr);
   w.unit_done = reinterpret_cast<int32_t*>(base + L.unit_done);
   w.att_cnt = reinterpret_cast<int32_t*>(base + L.att_cnt);
   w.ckey = reinterpret_cast<uint32_t*>(base + L.ckey);
   w.coff = reinterpret_cast<uint16_t*>(base + L.coff);
+  w.cpid = reinterpret_cast<int32_t*>(base + L.cpid);
   w.part = reinterpret_cast<float*>(base + L.part);
   w.g = persist_geom(p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
   w.units = p.B * p.Hkv;

@@ -30,6 +30,37 @@ __device__ __forceinline__ float key_score(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
+// NB bins over the keys in [lo, hi]: linear in the score between the smallest and the
+// largest one (scores near the top are then spread over many bins); when that range is not
+// finite, bins of width 2^sh in key space.  Either map is monotone in the key.
+template <int NB>
+struct KeyBinsT {
+  static constexpr int LOG2 = NB == 1024 ? 10 : (NB == 256 ? 8 : -1);
+  static_assert(LOG2 > 0, "1024 or 256 bins");
+  float flo, inv;
+  uint32_t lo;
+  int sh;
+  bool linear;
+  __device__ __forceinline__ KeyBinsT(uint32_t lo_, uint32_t hi) : lo(lo_) {
+    flo = key_score(lo_);
+    const float fhi = key_score(hi);
+    const float width = fhi - flo;
+    const float inv0 = __fdividef((float)NB, width);  // any positive scale is monotone
+    linear = isfinite(flo) && isfinite(fhi) && width > 0.0f && isfinite(inv0);
+    inv = linear ? inv0 : 0.0f;
+    const int bits = 32 - __clz(hi - lo_);
+    sh = bits > LOG2 ? bits - LOG2 : 0;
+  }
+  __device__ __forceinline__ int operator()(uint32_t key) const {
+    if (linear) {
+      const float x = (key_score(key) - flo) * inv;
+      return x >= (float)(NB - 1) ? NB - 1 : (int)x;  // x >= 0 by construction
+    }
+    return (int)((key - lo) >> sh);
+  }
+};
+using KeyBins = KeyBinsT<kTopkBins>;
+
 // Scratch in shared memory: hist[kTopkBins] ints, small[64] ints.
 template <int NT, typename Emit>
 __device__ void block_topk(const uint32_t* keys, int m, int k, int* hist, int* small, Emit emit) {
@@ -64,23 +95,7 @@ __device__ void block_topk(const uint32_t* keys, int m, int k, int* hist, int* s
     lo = min(lo, (uint32_t)small[w]);
     hi = max(hi, (uint32_t)small[NW + w]);
   }
-  // Bins linear in the score between the smallest and the largest one (scores near the
-  // top are then spread over many bins); when the range is not finite, bins of width 2^sh
-  // in key space.  Either map is monotone in the key.
-  const float flo = key_score(lo), fhi = key_score(hi);
-  const float width = fhi - flo;
-  const float inv0 = (float)kTopkBins / width;
-  const bool linear = isfinite(flo) && isfinite(fhi) && width > 0.0f && isfinite(inv0);
-  const float inv = linear ? inv0 : 0.0f;
-  const int bits = 32 - __clz(hi - lo);
-  const int sh = bits > 10 ? bits - 10 : 0;
-  auto bin_of = [&](uint32_t key) -> int {
-    if (linear) {
-      const float x = (key_score(key) - flo) * inv;
-      return x >= (float)(kTopkBins - 1) ? kTopkBins - 1 : (int)x;  // x >= 0 by construction
-    }
-    return (int)((key - lo) >> sh);
-  };
+  const KeyBins bin_of(lo, hi);
   // 2. histogram
   for (int j = tid; j < m; j += NT) atomicAdd(&hist[bin_of(keys[j])], 1);
   __syncthreads();
@@ -89,7 +104,7 @@ __device__ void block_topk(const uint32_t* keys, int m, int k, int* hist, int* s
     constexpr int BPL = kTopkBins / 32;
     int tot = 0;
 #pragma unroll
-    for (int i = 0; i < BPL; ++i) tot += hist[lane * BPL + i];
+    for (int i = 0; i < BPL; ++i) tot += hist[lane * BPL + ((i + lane) & (BPL - 1))];  // no bank conflicts
     int incl = tot;  // sum over lanes >= lane
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -217,6 +232,119 @@ __device__ void block_topk(const uint32_t* keys, int m, int k, int* hist, int* s
     tie_off += __popc(tb);
   }
   __syncthreads();
+}
+
+// Shared-memory scratch of small_topk (16-byte aligned): hist[HIST] ints that are ZERO on
+// entry (hist[kSmallBins] counts the members of the threshold bin), list[2 NT] (key, index)
+// pairs, cnt[2 NW] ints.
+constexpr int kSmallBins = 256;
+template <int NT>
+struct SmallTopk {
+  static constexpr int HIST = kSmallBins + 4;
+  static constexpr int LIST = HIST * 4;                 // byte offset of list
+  static constexpr int CNT = LIST + 2 * NT * 8;         // byte offset of cnt
+  static constexpr int BYTES = CNT + 2 * (NT / 32) * 4;
+};
+
+// Exact top-k of m <= 2 NT keys, ties going to the lowest index, with two block barriers
+// (three when the bin of the k-th largest key holds more keys than are still needed).
+// On entry keys[0, m) and the zeroed histogram are visible to every thread and lo / hi are
+// the smallest and the largest of the keys.  Thread t owns keys t and t + NT.  emit(j, pos)
+// receives the selected indices with their positions in ascending index order; no barrier
+// follows the emits.  Steps: one histogram of kSmallBins bins monotone in the key; every warp
+// finds the threshold bin B from it on its own (no barrier); keys above B are selected, and
+// the keys of B are all selected when B holds exactly the number still needed, otherwise
+// ranked among the members of B (by key, then index).
+template <int NT, typename Emit>
+__device__ __forceinline__ void small_topk(const uint32_t* keys, int m, int k, uint32_t lo,
+                                           uint32_t hi, unsigned char* scratch, Emit emit) {
+  constexpr int NW = NT / 32;
+  using S = SmallTopk<NT>;
+  int* hist = reinterpret_cast<int*>(scratch);
+  uint2* list = reinterpret_cast<uint2*>(scratch + S::LIST);
+  int* cnt = reinterpret_cast<int*>(scratch + S::CNT);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int j0 = tid, j1 = tid + NT;
+  if (k <= 0) return;
+  if (k >= m) {  // every key is selected
+    if (j0 < m) emit(j0, j0);
+    if (j1 < m) emit(j1, j1);
+    return;
+  }
+  const uint32_t k0 = j0 < m ? keys[j0] : 0u, k1 = j1 < m ? keys[j1] : 0u;
+  const KeyBinsT<kSmallBins> bins(lo, hi);
+  auto bin_of = [&](uint32_t key) { return min(max(bins(key), 0), kSmallBins - 1); };
+  const int b0 = j0 < m ? bin_of(k0) : -1, b1 = j1 < m ? bin_of(k1) : -1;
+  if (b0 >= 0) atomicAdd(&hist[b0], 1);
+  if (b1 >= 0) atomicAdd(&hist[b1], 1);
+  __syncthreads();
+  // threshold bin, found by every warp.  Lane l totals bins [8 l, 8 l + 8) (two 16-byte
+  // loads, the pair's order rotated so that no two lanes of a phase share banks); a suffix scan
+  // over the lanes finds the lane src holding the k-th key, and lanes 0..7 then split src's
+  // eight bins for a second suffix scan.
+  static_assert(kSmallBins == 8 * 32, "eight bins per lane");
+  const int4* h4 = reinterpret_cast<const int4*>(hist);
+  const int rot = (lane >> 2) & 1;
+  const int4 va = h4[2 * lane + rot], vb = h4[2 * lane + (rot ^ 1)];
+  const int tot = ((va.x + va.y) + (va.z + va.w)) + ((vb.x + vb.y) + (vb.z + vb.w));
+  int incl = tot;  // keys in the bins of lanes >= lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_down_sync(kFull, incl, o);
+    if (lane + o < 32) incl += y;
+  }
+  const int src = __ffs(__ballot_sync(kFull, incl - tot < k && k <= incl)) - 1;
+  const int above = __shfl_sync(kFull, incl - tot, src);
+  const int i8 = lane & 7;
+  const int cbin = hist[8 * src + i8];
+  int s8 = cbin;  // keys in src's bins >= i8
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    const int y = __shfl_down_sync(kFull, s8, o, 8);
+    if (i8 + o < 8) s8 += y;
+  }
+  const int bi = __ffs(__ballot_sync(kFull, lane < 8 && above + s8 - cbin < k && k <= above + s8)) - 1;
+  const int B = 8 * src + bi;
+  const int cntB = __shfl_sync(kFull, cbin, bi);
+  const int need = k - above - __shfl_sync(kFull, s8 - cbin, bi);
+  bool s0 = b0 > B, s1 = b1 > B;
+  if (cntB == need) {
+    s0 |= b0 == B;
+    s1 |= b1 == B;
+  } else {
+    if (b0 == B) list[atomicAdd(&hist[kSmallBins], 1)] = make_uint2(k0, (uint32_t)j0);
+    if (b1 == B) list[atomicAdd(&hist[kSmallBins], 1)] = make_uint2(k1, (uint32_t)j1);
+    __syncthreads();
+    auto ranked_in = [&](uint32_t key, int j) {
+      int r = 0;
+      for (int i = 0; i < cntB; ++i) {
+        const uint2 e = list[i];
+        r += (e.x > key) || (e.x == key && (int)e.y < j);
+      }
+      return r < need;
+    };
+    if (b0 == B) s0 = ranked_in(k0, j0);
+    if (b1 == B) s1 = ranked_in(k1, j1);
+  }
+  const unsigned bal0 = __ballot_sync(kFull, s0), bal1 = __ballot_sync(kFull, s1);
+  if (lane == 0) {
+    cnt[warp] = __popc(bal0);
+    cnt[NW + warp] = __popc(bal1);
+  }
+  __syncthreads();
+  int off0 = 0, off1 = 0, tot0 = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const int c0 = cnt[w];
+    tot0 += c0;
+    if (w < warp) {
+      off0 += c0;
+      off1 += cnt[NW + w];
+    }
+  }
+  const unsigned lt = (1u << lane) - 1u;
+  if (s0) emit(j0, off0 + __popc(bal0 & lt));
+  if (s1) emit(j1, tot0 + off1 + __popc(bal1 & lt));
 }
 
 // Reduce N per-lane partial sums over aligned groups of L lanes (N <= L, both powers of two)

@@ -156,8 +156,13 @@ def test_fused_workspace_reuse(name, oracle):
     assert int(st.item()) == 0
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
-    # the queue counters are back to zero after every call (epoch word aside)
-    assert int(ws[:12].count_nonzero()) == 0
+    # after a complete call the claim count equals the next launch's starting count, and the
+    # per-unit counters (after the first 256 bytes, B * Hkv int32 each, 256-byte aligned) are 0
+    head = ws[:8].view(torch.int32)
+    assert int(head[0]) == int(head[1]) > 0
+    units = c.B * c.Hkv
+    span = 2 * ((units * 4 + 255) // 256 * 256)
+    assert int(ws[256:256 + span].count_nonzero()) == 0
 
 
 def test_planner_order_and_invariance(oracle):
