@@ -43,7 +43,8 @@ constexpr int kPersistThreads = 128;
 constexpr int kPersistWarps = kPersistThreads / 32;
 constexpr int kChunk = 256;      // candidate pages per scan item (64 per warp)
 constexpr int kScanRing = 4;     // 8-row centroid batches per warp ring (3 landing)
-constexpr int kPiecePages = 16;  // most selected pages per attention item (4 per warp)
+constexpr int kPiecePages = 32;  // most selected pages per attention item (8 per warp)
+constexpr int kTailPiecePages = 16;  // the same for the later half of the units
 constexpr int kMaxPlanB = 2048;  // requests the persistent path takes (schedule kept in smem)
 constexpr int kPersistMinCtas = 3;  // CTAs per SM the registers must allow (<= 168 per thread)
 
@@ -53,8 +54,10 @@ struct PersistGeom {
   int max_cand;  // middle (candidate) pages of a full page-table row, >= 1
   int nch_max;   // chunks of such a row
   int kc;        // candidates a chunk keeps: min(topk, kChunk)
-  int A;         // attention pieces per unit
-  int pp;        // selected pages per piece: kmax split evenly, at most kPiecePages
+  int A;         // attention pieces of each of the earlier half of the units
+  int pp;        // their selected pages per piece: kmax split evenly, at most kPiecePages
+  int A2, pp2;   // the same for the later half (at most kTailPiecePages): their attention
+                 // runs at the end of the launch, where more, shorter items keep more CTAs busy
   int cmax;      // candidates one unit merges at most
 };
 
@@ -67,6 +70,8 @@ __host__ __device__ inline PersistGeom persist_geom(int64_t pt_stride, int topk,
   g.kc = topk < kChunk ? (topk > 0 ? topk : 1) : kChunk;
   g.A = (kmax + kPiecePages - 1) / kPiecePages;
   g.pp = (kmax + g.A - 1) / g.A;
+  g.A2 = (kmax + kTailPiecePages - 1) / kTailPiecePages;
+  g.pp2 = (kmax + g.A2 - 1) / g.A2;
   const int64_t c = (int64_t)g.nch_max * g.kc;
   g.cmax = c < g.max_cand ? (int)c : g.max_cand;
   return g;
@@ -90,7 +95,7 @@ struct PersistWs {
   uint32_t* ckey;      // [U][nch_max][kc]: ordered score keys of each chunk's top-k
   uint16_t* coff;      // [U][nch_max][kc]: their offsets in the chunk, ascending
   int32_t* cpid;       // [U][nch_max][kc]: their page ids (-1 where the id was out of range)
-  float* part;         // [U][A][G][Dv+2]: attention partials
+  float* part;         // [U][A2][G][Dv+2]: attention partials
   PersistGeom g;
   int units;
 };
@@ -117,7 +122,7 @@ static PersistWsLayout persist_ws_layout(const DecodeParams& p, int G, int Dv, i
   L.ckey = o;      o += align256(cand * sizeof(uint32_t));
   L.coff = o;      o += align256(cand * sizeof(uint16_t));
   L.cpid = o;      o += align256(cand * sizeof(int32_t));
-  L.part = o;      o += align256(U * g.A * G * (Dv + 2) * sizeof(float));
+  L.part = o;      o += align256(U * g.A2 * G * (Dv + 2) * sizeof(float));
   L.total = o;
   return L;
 }
@@ -168,7 +173,7 @@ __host__ __device__ inline PersistSmem persist_smem_layout(int D, int G, int B,
   const int merge_big = align16(g.cmax * 4) + align16(g.cmax * 2) + align16((kTopkBins + 64) * 4);
   const int merge = merge_small > merge_big ? merge_small : merge_big;
   const int comb = align16(kPersistWarps * G * (D + 2) * 4) + align16(G * (D + 2) * 4) +
-                   align16(g.A * G * (D + 2) * 4);
+                   align16(g.A2 * G * (D + 2) * 4);
   int r = scan;
   if (att > r) r = att;
   if (merge > r) r = merge;
@@ -192,7 +197,6 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
 
   extern __shared__ __align__(128) unsigned char smem[];
   const PersistGeom gm = w.g;
-  const int A = gm.A;
   const PersistSmem Ls = persist_smem_layout(D, G, p.B, gm);
   int* s_prefix = reinterpret_cast<int*>(smem + Ls.prefix);
   uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem + Ls.keys);
@@ -252,7 +256,8 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
     __syncthreads();
   }
   const int scan_items = s_prefix[p.B];
-  const int total_items = scan_items + w.units * A;
+  const int u_split = w.units / 2;  // units from here on take gm.A2 pieces
+  const int total_items = scan_items + u_split * gm.A + (w.units - u_split) * gm.A2;
 
   // A counter that thread 0 bumps (release) once the CTA has passed the barrier at the end
   // of the item that produced the counted data, so that the fence overlaps the next item.
@@ -318,9 +323,9 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
       }
       if (lane < myrows) s_pids[warp + NW * lane] = pidA;
       if (lane + 32 < myrows) s_pids[warp + NW * (lane + 32)] = pidB;
-      const uint32_t ring = region_u32 + warp * kScanRing * 8 * S::C_ROW;
       const float* cbase = p.centroids + (int64_t)h * D;
       const int64_t cstride = (int64_t)p.Hkv * D;
+      const uint32_t ring = region_u32 + warp * kScanRing * 8 * S::C_ROW;
       const int batches = (myrows + 7) / 8;
       constexpr int CPRS = S::C_ROW / 16;  // 16-byte chunks per centroid row
       auto issue = [&](int bt) {
@@ -406,7 +411,10 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
     } else {
       // ---------------------------------------------------------------- attention item
       const int a = t - scan_items;
-      const int u = a / A, piece = a - u * A;
+      const bool early = a < u_split * gm.A;
+      const int A = early ? gm.A : gm.A2, pp = early ? gm.pp : gm.pp2;
+      const int a2 = early ? a : a - u_split * gm.A;
+      const int u = (early ? 0 : u_split) + a2 / A, piece = a2 % A;
       const int b = u / p.Hkv, h = u - b * p.Hkv;
       const int L = p.seq_lens[b];
       const int n = (L + kPage - 1) / kPage;
@@ -414,8 +422,8 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
       const bool dense = n <= p.kmax;
       const int nch = chunks_of(L, p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
       const int ns = !valid ? 0 : (dense ? n : p.kmax);
-      const int j0 = piece * gm.pp;
-      const int np = max(0, min(ns - j0, gm.pp));
+      const int j0 = piece * pp;
+      const int np = max(0, min(ns - j0, pp));
       const bool write_sel = piece == 0 && p.sel != nullptr;
       int32_t* selrow = write_sel ? p.sel + (int64_t)u * p.kmax : nullptr;
       if (tid == 0 && piece == 0) {
@@ -592,7 +600,7 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
         if (A > 1) {
           if (piece < A - 1) {
             // publish this piece's partial and move on: the unit's last piece merges them
-            float* dst = w.part + ((int64_t)u * A + piece) * G * (D + 2);
+            float* dst = w.part + ((int64_t)u * gm.A2 + piece) * G * (D + 2);
             for (int i = tid; i < G * (D + 2); i += NT) dst[i] = s_cp[i];
             pending = w.att_cnt + u;
             fin = 0;
@@ -618,7 +626,7 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
             __syncthreads();
             fin = s_misc[1];
             if (fin) {
-              const float* src = w.part + (int64_t)u * A * G * (D + 2);
+              const float* src = w.part + (int64_t)u * gm.A2 * G * (D + 2);
               for (int i = tid; i < (A - 1) * G * (D + 2); i += NT) s_all[i] = __ldcg(src + i);
               for (int i = tid; i < G * (D + 2); i += NT) s_all[(A - 1) * G * (D + 2) + i] = s_cp[i];
               __syncthreads();
