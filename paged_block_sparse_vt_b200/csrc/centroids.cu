@@ -18,6 +18,11 @@ __global__ void __launch_bounds__(256) build_centroids_kernel(
     const __nv_bfloat16* __restrict__ k_pool, int64_t num_pages, int num_kv_heads, int head_dim,
     int64_t sk_p, int64_t sk_t, int64_t sk_h, const int32_t* __restrict__ pages, int n_pages,
     float* __restrict__ centroids, int32_t* status) {
+  // Launched as a programmatic dependent of the previous kernel on the stream (which may read
+  // the centroids): nothing is read or written before that kernel has completed.  The next
+  // kernel may be placed at once and waits the same way.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   const int chunks = head_dim >> 3;
   const int64_t per_page = (int64_t)num_kv_heads * chunks;
   const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -59,10 +64,20 @@ cudaError_t launch_build_centroids(const vt_paged_kv& kv, const int32_t* pages, 
   if (threads == 0) return cudaSuccess;
   const int nt = 256;
   const int64_t blocks = (threads + nt - 1) / nt;
-  build_centroids_kernel<<<(unsigned)blocks, nt, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(kv.k_pool), kv.num_pages, kv.num_kv_heads, kv.head_dim,
-      kv.sk_p, kv.sk_t, kv.sk_h, pages, n_pages, centroids, status);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(nt);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, build_centroids_kernel,
+                            static_cast<const __nv_bfloat16*>(kv.k_pool), kv.num_pages,
+                            kv.num_kv_heads, kv.head_dim, kv.sk_p, kv.sk_t, kv.sk_h, pages,
+                            n_pages, centroids, status);
 }
 
 }  // namespace vt
