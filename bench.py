@@ -71,13 +71,14 @@ def algorithmic_bytes(c, seq_lens: torch.Tensor) -> dict:
     sel_pages = torch.minimum(n, torch.full_like(n, c.kmax))
     tokens = PAGE_SIZE * (sel_pages - 1) + last_valid
     per_req = 2 * c.Hq * c.D + 2 * c.Hq * c.Dv + 4 * c.Hq + 4 * n
-    per_unit = 4 * c.D * cand + 2 * (c.D + c.Dv) * tokens
+    dv = 0 if c.mla else c.Dv  # MLA: V is the first Dv dims of the K row, read once
+    per_unit = 4 * c.D * cand + 2 * (c.D + dv) * tokens
     fused = int(per_req.sum()) + c.Hkv * int(per_unit.sum())
     n_fill = int((L % PAGE_SIZE == 0).sum())
     build = n_fill * (PAGE_SIZE * c.Hkv * c.D * 2 + c.Hkv * c.D * 4 + 4)
     return dict(fused=fused, build=build, total=fused + build,
                 centroid_bytes=c.Hkv * int((4 * c.D * cand).sum()),
-                kv_bytes=c.Hkv * int((2 * (c.D + c.Dv) * tokens).sum()))
+                kv_bytes=c.Hkv * int((2 * (c.D + dv) * tokens).sum()))
 
 
 def read_peak_hbm():
@@ -256,8 +257,8 @@ def run_reference(args, world, rank):
     if rank != 0:
         return  # rank 0 alone runs the CPU reference
     import oracle
-    c = config(CFG)
-    w = make_workload(c)
+    c = config(args.config)
+    w = make_workload(c, seed=1000 + args.config)
     cent = oracle_prepare(w)
     cores = oracle.get_threads()
     reqs = oracle_sample_size(w, cent, target_s=max(0.5, 60.0 / max(1, args.steps + args.warmup)))
@@ -283,10 +284,19 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def lengths_text(c) -> str:
+    if c.lengths == "fixed":
+        return f"{c.len_lo}"
+    if c.lengths == "uniform":
+        return f"U[{c.len_lo},{c.len_hi}]"
+    return f"logU[{c.len_lo},{c.len_hi}]"
+
+
 def workload_config(c, w, args) -> dict:
     return {
-        "workload": f"qwen3-0.6b-like sparse decode layer (B={c.B}, Hq={c.Hq}, Hkv={c.Hkv}, "
-                    f"D={c.D}, page 16, context U[{c.len_lo},{c.len_hi}], top-{c.topk}+{c.bos}+{c.eos})",
+        "workload": f"{c.name} sparse decode layer (B={c.B}, Hq={c.Hq}, Hkv={c.Hkv}, "
+                    f"D={c.D}/{c.Dv}, page 16, context {lengths_text(c)}, "
+                    f"top-{c.topk}+{c.bos}+{c.eos})",
         "B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "head_dim": c.D, "page_size": PAGE_SIZE,
         "topk": c.topk, "bos": c.bos, "eos": c.eos, "pool_pages": w["P"],
         "mean_pages_per_request": float(((w["seq_lens"].double() + 15) // 16).mean()),
@@ -303,16 +313,18 @@ def run_ours(args, world, rank, local):
     vt.load_library()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    c = config(CFG)
-    w = make_workload(c, seed=1000 + CFG + 7919 * rank)
+    c = config(args.config)
+    w = make_workload(c, seed=1000 + args.config + 7919 * rank)
     nbytes = algorithmic_bytes(c, w["seq_lens"])
     stream = torch.cuda.current_stream(dev)
 
     # resident replicas of every per-step input; centroids of the full pages prebuilt
     reps = []
     for r in range(args.replicas):
-        d = {k: w[k].to(dev) for k in ("q", "k_pool", "v_pool", "page_table", "seq_lens",
+        d = {k: w[k].to(dev) for k in ("q", "k_pool", "page_table", "seq_lens",
                                         "prebuilt_pages", "fill_pages")}
+        # MLA: V is a view of the K rows (one pool)
+        d["v_pool"] = d["k_pool"] if w["v_pool"] is w["k_pool"] else w["v_pool"].to(dev)
         d["cent"] = torch.zeros((w["P"], c.Hkv, c.D), dtype=torch.float32, device=dev)
         vt.vt_build_centroids(d["k_pool"], d["prebuilt_pages"], d["cent"])
         d["out"] = torch.empty((c.B, c.Hq, c.Dv), dtype=torch.bfloat16, device=dev)
@@ -320,7 +332,8 @@ def run_ours(args, world, rank, local):
         d["order"] = torch.empty((c.B,), dtype=torch.int32, device=dev)
         d["status"] = torch.zeros((1,), dtype=torch.int32, device=dev)
         d["ws"] = vt.fused_workspace(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
-                                     d["seq_lens"], d["cent"], c.topk, c.bos, c.eos)
+                                     d["seq_lens"], d["cent"], c.topk, c.bos, c.eos,
+                                     head_dim_v=c.Dv)
         reps.append(d)
     torch.cuda.synchronize(dev)
 
@@ -329,7 +342,7 @@ def run_ours(args, world, rank, local):
                                   d["seq_lens"], d["cent"], c.topk, c.bos, c.eos, c.sm_scale,
                                   out=d["out"], lse=d["lse"],
                                   order=d["order"] if args.plan else None, status=d["status"],
-                                  workspace=d["ws"])
+                                  workspace=d["ws"], head_dim_v=c.Dv)
 
     def step(d):
         vt.vt_build_centroids(d["k_pool"], d["fill_pages"], d["cent"], status=d["status"])
@@ -469,6 +482,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--replicas", type=int, default=3)
+    ap.add_argument("--config", type=int, default=CFG, choices=[1, 2, 3, 4, 5],
+                    help="workload of the hot-path table (the headline line is config 2)")
     ap.add_argument("--plan", action="store_true",
                     help="add the vt_plan_requests launch to the step")
     ap.add_argument("--no-cpu-baseline", action="store_true")

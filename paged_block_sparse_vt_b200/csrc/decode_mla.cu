@@ -30,10 +30,13 @@ constexpr int kMlaD = 576;
 constexpr int kMlaDv = 512;
 constexpr int kMlaRow = kMlaD + 8;  // smem row stride (elements): 1168 B, ldmatrix conflict-free
 constexpr int kMlaMaxPages = 8;     // pages one CTA attends to (one warp per page)
+constexpr int kMlaScanRows = 2;     // centroid rows per ring slot (2 x 2304 B)
+constexpr int kMlaScanSlots = 4;    // ring slots per warp: 3 batches landing while one is used
+constexpr int kMlaRingBytes = (kMlaThreads / 32) * kMlaScanSlots * kMlaScanRows * kMlaD * 4;
 
 struct MlaSmem {
   int sel, phys, misc;               // persistent
-  int qm, cpage, score, key;         // selection phase
+  int qm, cpage, score, key, ring;   // selection phase
   int q, kt, st, pm, ml;             // attention phase (aliases the selection phase)
   int total;
 };
@@ -51,6 +54,7 @@ __host__ __device__ inline MlaSmem mla_smem_layout(int G, int cand_cap, int key_
   s.cpage = a; a += align16(cand_cap * 4);
   s.score = a; a += align16(cand_cap * 4);
   s.key = a;   a += align16(key_cap * 4);
+  s.ring = a;  a += kMlaRingBytes;  // per-warp cp.async rings of centroid rows
   int b = base;  // attention phase
   const int T = ppc * kPage;
   s.q = b;  b += align16(G * kMlaRow * 2);
@@ -71,7 +75,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const Decode
   constexpr int NW = NT / 32;
   constexpr int D = kMlaD, DV = kMlaDv;
   constexpr int CH = D / 4;  // float4 per centroid row (144)
-  constexpr int US = 2;      // centroid rows per warp in flight
   static_assert(G == 16 || G == 32, "MLA path: 16 or 32 query heads");
 
   extern __shared__ __align__(16) unsigned char smem[];
@@ -159,44 +162,70 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const Decode
       }
       if (__syncthreads_or(badp) && tid == 0) flag(p.status, VT_DEV_BAD_PAGE);
       {
-        // one warp per centroid row, float4 chunks ch = lane + 32 i (i < 5; the 5th only for
-        // lanes < 16), US rows in flight per warp
+        // Warp w scores rows w + NW i of the CTA's candidates: the fp32 centroid rows stream
+        // through the warp's ring of kMlaScanSlots slots of kMlaScanRows rows (cp.async, three
+        // slots landing while one is used); float4 chunk c = lane + 32 i of a row (i < 5, the
+        // 5th only for lanes < 16) is dotted with the same chunk of the group mean.
         float4 qv[5];
 #pragma unroll
         for (int i = 0; i < 5; ++i) {
           const int c = lane + 32 * i;
           qv[i] = c < CH ? reinterpret_cast<const float4*>(s_qm)[c] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        for (int r0 = warp; r0 < cnt; r0 += NW * US) {
-          float4 cv[US][5];
+        constexpr int RB = D * 4;  // bytes of a centroid row
+        const uint32_t ring = smem_u32(smem + Ls.ring) + warp * kMlaScanSlots * kMlaScanRows * RB;
+        const int myrows = (cnt - warp + NW - 1) / NW;
+        const int nb = (myrows + kMlaScanRows - 1) / kMlaScanRows;
+        auto issue = [&](int bt) {
+          if (bt < nb) {
+            const uint32_t dst = ring + (bt % kMlaScanSlots) * kMlaScanRows * RB;
 #pragma unroll
-          for (int u = 0; u < US; ++u) {
-            const int r = r0 + u * NW;
-            const int pg = r < cnt ? s_cpage[r] : -1;
-            const float* row = p.centroids + (int64_t)(pg < 0 ? 0 : pg) * D;
-#pragma unroll
-            for (int i = 0; i < 5; ++i) {
-              const int c = lane + 32 * i;
-              cv[u][i] = (pg >= 0 && c < CH) ? ld_stream_f4(row + 4 * c)
-                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int rr = 0; rr < kMlaScanRows; ++rr) {
+              const int i = bt * kMlaScanRows + rr;
+              const int pg = i < myrows ? s_cpage[warp + NW * i] : -1;
+              if (pg >= 0) {
+                const float* row = p.centroids + (int64_t)pg * D;
+                for (int c = lane; c < CH; c += 32) cp_async16(dst + rr * RB + c * 16, row + 4 * c, 16);
+              }
             }
           }
+          cp_async_commit();
+        };
 #pragma unroll
-          for (int u = 0; u < US; ++u) {
+        for (int bt = 0; bt < kMlaScanSlots - 1; ++bt) issue(bt);
+        for (int bt = 0; bt < nb; ++bt) {
+          issue(bt + kMlaScanSlots - 1);
+          cp_async_wait<kMlaScanSlots - 1>();
+          __syncwarp();
+          const uint32_t src = ring + (bt % kMlaScanSlots) * kMlaScanRows * RB;
+#pragma unroll
+          for (int rr = 0; rr < kMlaScanRows; ++rr) {
             float d = 0.0f;
 #pragma unroll
             for (int i = 0; i < 5; ++i) {
-              d = fmaf(cv[u][i].x, qv[i].x, d);
-              d = fmaf(cv[u][i].y, qv[i].y, d);
-              d = fmaf(cv[u][i].z, qv[i].z, d);
-              d = fmaf(cv[u][i].w, qv[i].w, d);
+              const int c = lane + 32 * i;
+              if (c < CH) {
+                float4 cv;
+                asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+                             : "=f"(cv.x), "=f"(cv.y), "=f"(cv.z), "=f"(cv.w)
+                             : "r"(src + rr * RB + c * 16));
+                d = fmaf(cv.x, qv[i].x, d);
+                d = fmaf(cv.y, qv[i].y, d);
+                d = fmaf(cv.z, qv[i].z, d);
+                d = fmaf(cv.w, qv[i].w, d);
+              }
             }
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) d += __shfl_xor_sync(kFull, d, o);
-            const int r = r0 + u * NW;
-            if (lane == 0 && r < cnt) s_score[r] = (s_cpage[r] >= 0) ? d : -INFINITY;
+            const int i = bt * kMlaScanRows + rr;
+            if (lane == 0 && i < myrows) {
+              const int r = warp + NW * i;
+              s_score[r] = (s_cpage[r] >= 0) ? d : -INFINITY;
+            }
           }
+          __syncwarp();  // every lane is done with the slot before it is refilled
         }
+        cp_async_wait<0>();
       }
       cluster.sync();  // #1
       if (rank == 0) {
