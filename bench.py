@@ -103,12 +103,13 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic():
-    """DRAM bytes per launch of the fused kernel from an ncu capture, if taken on this source."""
+def recorded_traffic(cfg: int):
+    """DRAM bytes per launch of the fused kernel from an ncu capture, if it was taken on this
+    source and this workload."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
-        if rec.get("source_hash") == kernel_source_hash():
+        if rec.get("source_hash") == kernel_source_hash() and rec.get("config", CFG) == cfg:
             return rec.get("bytes_per_launch")
     except Exception:
         pass
@@ -435,8 +436,9 @@ def run_ours(args, world, rank, local):
         "config": workload_config(c, w, args),
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "traffic": recorded_traffic(),
-            "kernel": "persist_fused_kernel (vt_sparse_decode_fused)",
+            "frac": achieved / peak, "traffic": recorded_traffic(args.config),
+            "kernel": ("persist_mla_kernel" if c.mla else "persist_fused_kernel")
+                      + " (vt_sparse_decode_fused)",
             "algorithmic_bytes_per_launch": nbytes["fused"], "kernel_ms": fused_ms,
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
             else "fallback 6650 GB/s",

@@ -161,17 +161,18 @@ vt_status vt_sparse_decode(const vt_paged_kv* kv, const vt_decode_args* a, const
  * within that rounding of each other, which of them is kept).  sel / n_sel
  * receive the selection when not NULL (both or neither).
  *
- * For GQA heads with B <= 2048 the work runs as one launch of persistent
- * CTAs fed from a queue of small scan and attention items that the CTAs
- * derive from seq_lens themselves (a->order is not used there), which keeps
- * every SM busy on batches of very uneven lengths; it needs `workspace`: device memory of vt_fused_workspace_size()
+ * For B <= 2048 the work runs as one launch of persistent CTAs fed from a
+ * queue of small scan and attention items that the CTAs derive from seq_lens
+ * themselves (a->order is not used there), which keeps every SM busy on
+ * batches of very uneven lengths; it needs `workspace`: device memory of vt_fused_workspace_size()
  * bytes, 256-byte aligned, ZERO-FILLED ONCE when allocated.  Every call
  * leaves it ready for the next one with the same B * Hkv, so it is zeroed
  * only once (its counter arrays are laid out for B * Hkv units: zero it again
  * before a call with another B * Hkv).  Calls that share a workspace must not
  * overlap on the GPU (use one stream, or one workspace per stream); after a
- * call that reported VT_DEV_TIMEOUT, zero it again.  When vt_fused_workspace_size() is 0 (MLA, or B > 2048) no
- * workspace is used and `workspace` may be NULL.
+ * call that reported VT_DEV_TIMEOUT, zero it again.  When
+ * vt_fused_workspace_size() is 0 (B > 2048) no workspace is used and
+ * `workspace` may be NULL.
  */
 vt_status vt_sparse_decode_fused(const vt_paged_kv* kv, const vt_decode_args* a, void* out,
                                  float* lse, int32_t* sel, int32_t* n_sel, void* workspace,
@@ -200,7 +201,7 @@ size_t vt_fused_workspace_size(const vt_paged_kv* kv, const vt_decode_args* a);
  * zero again; the candidate and partial arrays after them are always written
  * before they are read.  A call whose vt_fused_workspace_size() exceeds
  * VT_STATIC_SCRATCH_BYTES fails with VT_ERR_UNSUPPORTED before anything is
- * launched; shapes that need no workspace (MLA, B > 2048) run as
+ * launched; shapes that need no workspace (B > 2048) run as
  * vt_sparse_decode_fused does.
  *
  * Races: every call on one device shares the one scratch.  Two calls that can

@@ -21,6 +21,11 @@ cudaError_t launch_plan(const int32_t* seq_lens, int B, int32_t* order, cudaStre
 size_t persist_workspace_bytes(const DecodeParams& p, int G, int Dv, int64_t unit_cap);
 int persist_smem_bytes(const DecodeParams& p, int D, int G);
 int persist_max_batch();
+size_t mla_persist_workspace_bytes(const DecodeParams& p, int G, int64_t unit_cap);
+int mla_persist_smem_bytes(const DecodeParams& p, int G);
+int mla_persist_max_batch();
+cudaError_t launch_mla_persist(const DecodeParams& p, int G, void* ws, int64_t unit_cap,
+                               int sm_count, cudaStream_t s);
 cudaError_t launch_persist_fused(const DecodeParams& p, int D, int G, void* ws, int64_t unit_cap,
                                  int sm_count, cudaStream_t s);
 }  // namespace vt
@@ -190,9 +195,17 @@ vt_status fill_params(const vt_paged_kv* kv, const vt_decode_args* a, bool need_
   return ok();
 }
 
-// The fused GQA call runs on persistent CTAs (needs a workspace) up to this many requests.
+// The fused call runs on persistent CTAs (and needs a workspace) up to this many requests.
 bool use_persistent(const Shape& sh, const vt_decode_args* a) {
-  return sh.path == kPathGqa && a->batch >= 1 && a->batch <= persist_max_batch();
+  if (a->batch < 1) return false;
+  if (sh.path == kPathMla) return a->batch <= mla_persist_max_batch();
+  return sh.path == kPathGqa && a->batch <= persist_max_batch();
+}
+
+// Workspace of the persistent fused path (its counters laid out for unit_cap units, 0: B*Hkv).
+size_t persist_bytes(const Shape& sh, const DecodeParams& p, int64_t unit_cap) {
+  return sh.path == kPathMla ? mla_persist_workspace_bytes(p, sh.G, unit_cap)
+                             : persist_workspace_bytes(p, sh.G, sh.Dv, unit_cap);
 }
 
 // unit_cap: units the persistent path's counter arrays are laid out for (0: exactly B * Hkv)
@@ -215,15 +228,18 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
   p.lse = lse;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (mode == kFused && use_persistent(sh, a)) {
-    const size_t need = persist_workspace_bytes(p, sh.G, sh.Dv, unit_cap);
+    const size_t need = persist_bytes(sh, p, unit_cap);
     if (!ws || ws_bytes < need)
       return fail(VT_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need,
                   ws ? ws_bytes : (size_t)0);
     if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
       return fail(VT_ERR_INVALID_ARG, "workspace not 256-byte aligned");
-    const int bytes = persist_smem_bytes(p, sh.D, sh.G);
+    const int bytes = sh.path == kPathMla ? mla_persist_smem_bytes(p, sh.G)
+                                          : persist_smem_bytes(p, sh.D, sh.G);
     if (bytes > 227 * 1024) return fail(VT_ERR_UNSUPPORTED, "shared memory need %d B too large", bytes);
-    cudaError_t e = launch_persist_fused(p, sh.D, sh.G, ws, unit_cap, sm_count(), st);
+    cudaError_t e = sh.path == kPathMla
+                        ? launch_mla_persist(p, sh.G, ws, unit_cap, sm_count(), st)
+                        : launch_persist_fused(p, sh.D, sh.G, ws, unit_cap, sm_count(), st);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return ok();
   }
@@ -322,7 +338,7 @@ size_t vt_fused_workspace_size(const vt_paged_kv* kv, const vt_decode_args* a) {
   DecodeParams p;
   if (fill_params(kv, a, true, &sh, &p) != VT_OK) return 0;
   if (!use_persistent(sh, a)) return 0;
-  return persist_workspace_bytes(p, sh.G, sh.Dv, 0);
+  return persist_bytes(sh, p, 0);
 }
 
 vt_status vt_sparse_decode_fused_static(const vt_paged_kv* kv, const vt_decode_args* a,
@@ -338,7 +354,7 @@ vt_status vt_sparse_decode_fused_static(const vt_paged_kv* kv, const vt_decode_a
       if ((int64_t)a->batch * kv->num_kv_heads > kStaticUnitCap)
         return fail(VT_ERR_UNSUPPORTED, "B * Hkv > %lld units for the static scratch",
                     (long long)kStaticUnitCap);
-      need = persist_workspace_bytes(p, sh.G, sh.Dv, kStaticUnitCap);
+      need = persist_bytes(sh, p, kStaticUnitCap);
     }
   }
   if (need > (size_t)VT_STATIC_SCRATCH_BYTES)

@@ -1,0 +1,885 @@
+// fused_mla_persistent.cu -- the fused query side for the MLA latent form (one shared latent
+// KV head, K row = [latent 512 ; rope 64] bf16, V = the latent part of the same row, 16 or 32
+// absorbed query heads of 576 dims) on persistent CTAs that pull work items from a queue.
+//
+// Sources: "Vortex: Efficient and Programmable Sparse Attention Serving for AI Agents"
+// (rndamp.com), "Speedups that scale to 229B parameters" (rope-aware block sparse attention for
+// the MLA-based GLM-4.7-Flash on B200) and "A dual-stage programmable abstraction" (workload
+// planner, kernel fusion); the thread on digg.com, part [4/6] (MLA's shared latent); the flow
+// itself as in the vortex_torch README "Quick Example".  Rope-aware scoring
+// q_lat . c_lat + q_rope . c_rope is one dot product over the 576-dim row (the page mean is
+// linear in each part).
+//
+// One CTA of 8 warps per SM (the attention stages Q and eight K tiles: ~210 KB).  Items:
+//   scan items   -- (request, chunk of kMlaChunk candidate pages): each warp streams its rows
+//                   of fp32 centroids (2304 B each) through a cp.async ring and dots them with
+//                   the fp32 mean of the request's query heads; the CTA keeps the chunk's exact
+//                   top-k (key, offset, page id) and counts the chunk done;
+//   attention    -- (request, piece of <= 8 selected pages): waits until every chunk of the
+//   items           request is counted, merges the chunks' candidates with the same exact
+//                   top-k, stages Q and the piece's K tiles once in shared memory and runs
+//                   S^T = K Q^T (one warp per page), the softmax over the piece's tokens and
+//                   O = P V (each warp owns 64 of the 512 output dims) on the tensor cores;
+//                   with several pieces, the last one waits for the others' partials in the
+//                   workspace and merges them in registers.
+// Queue, claims and counters work as in the GQA persistent kernel (fused_persistent.cu).
+#include "decode_params.cuh"
+#include "topk.cuh"
+
+namespace vt {
+
+constexpr int kMpThreads = 256;
+constexpr int kMpWarps = kMpThreads / 32;
+constexpr int kMpD = 576;
+constexpr int kMpDv = 512;
+constexpr int kMpRow = kMpD + 8;   // smem row stride of Q and K tiles (elements): conflict-free ldmatrix
+constexpr int kMlaChunk = 128;     // candidate pages per scan item (16 per warp)
+constexpr int kMpScanRows = 2;     // centroid rows per ring slot
+constexpr int kMpScanSlots = 5;    // ring slots per warp (4 landing while one is used)
+constexpr int kMpPiece = 8;        // most selected pages per attention item (one warp each)
+constexpr int kMpMaxB = 2048;      // requests the persistent path takes
+
+// ---- sizes derived from the call ----------------------------------------------------------
+
+struct MpGeom {
+  int max_cand;  // middle (candidate) pages of a full page-table row, >= 1
+  int nch_max;   // chunks of such a row
+  int kc;        // candidates a chunk keeps: min(topk, kMlaChunk)
+  int cmax;      // candidates one request merges at most
+  int A, pp;     // attention pieces per request and their selected pages
+};
+
+__host__ __device__ inline MpGeom mp_geom(int64_t pt_stride, int topk, int bos, int eos, int kmax) {
+  MpGeom g;
+  const int64_t mc = pt_stride - bos - eos;
+  g.max_cand = mc > 1 ? (int)mc : 1;
+  g.nch_max = (g.max_cand + kMlaChunk - 1) / kMlaChunk;
+  g.kc = topk < kMlaChunk ? (topk > 0 ? topk : 1) : kMlaChunk;
+  const int64_t c = (int64_t)g.nch_max * g.kc;
+  g.cmax = c < g.max_cand ? (int)c : g.max_cand;
+  g.A = (kmax + kMpPiece - 1) / kMpPiece;
+  g.pp = (kmax + g.A - 1) / g.A;
+  return g;
+}
+
+// scan items of one request: none when nothing is ranked, else one per chunk of candidates
+__host__ __device__ inline int mp_chunks(int L, int64_t pt_stride, int topk, int bos, int eos,
+                                         int kmax) {
+  const int n = (L + kPage - 1) / kPage;
+  if (L < 1 || n > pt_stride || n <= kmax || topk < 1) return 0;
+  return (n - bos - eos + kMlaChunk - 1) / kMlaChunk;
+}
+
+struct MpWs {
+  uint32_t* ctr;       // [2]: claims ever made (mod 2^32), the count when this launch began
+  int32_t* unit_done;  // [B]: chunks of the request whose candidates are stored
+  int32_t* att_cnt;    // [B]: attention pieces of the request done
+  uint32_t* ckey;      // [B][nch_max][kc]: ordered score keys of each chunk's top-k
+  uint16_t* coff;      // [B][nch_max][kc]: their offsets in the chunk, ascending
+  int32_t* cpid;       // [B][nch_max][kc]: their page ids (-1 where out of range)
+  float* part;         // [B][A][G][Dv+2]: attention partials (acc, max, sum; base-2 max)
+  MpGeom g;
+};
+
+struct MpWsLayout {
+  size_t ctr, unit_done, att_cnt, ckey, coff, cpid, part, total;
+};
+
+static inline size_t mp_align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static MpWsLayout mp_ws_layout(const DecodeParams& p, int G, int64_t unit_cap) {
+  const MpGeom g = mp_geom(p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
+  const size_t U = (size_t)p.B;
+  const size_t cap = unit_cap > (int64_t)U ? (size_t)unit_cap : U;
+  const size_t cand = U * g.nch_max * g.kc;
+  MpWsLayout L;
+  size_t o = 0;
+  L.ctr = o;       o += mp_align256(2 * sizeof(uint32_t));
+  L.unit_done = o; o += mp_align256(cap * sizeof(int32_t));
+  L.att_cnt = o;   o += mp_align256(cap * sizeof(int32_t));
+  L.ckey = o;      o += mp_align256(cand * sizeof(uint32_t));
+  L.coff = o;      o += mp_align256(cand * sizeof(uint16_t));
+  L.cpid = o;      o += mp_align256(cand * sizeof(int32_t));
+  L.part = o;      o += mp_align256(U * g.A * G * (kMpDv + 2) * sizeof(float));
+  L.total = o;
+  return L;
+}
+
+// ---- shared memory -------------------------------------------------------------------------
+
+struct MpSmem {
+  int prefix, keys, pids, qm, sel, phys, ml, misc, region;  // region: one phase at a time
+  int ring, q, kt, pm, pmax, psum;                          // region offsets
+  int total;
+};
+
+__host__ __device__ inline MpSmem mp_smem_layout(int G, int B, const MpGeom& g) {
+  MpSmem s;
+  int o = 0;
+  s.prefix = o; o += align16((B + 1) * 4);
+  s.keys = o;   o += align16(kMlaChunk * 4);
+  s.pids = o;   o += align16(kMlaChunk * 4);
+  s.qm = o;     o += align16(kMpD * 4);
+  s.sel = o;    o += align16(kMpPiece * 4);
+  s.phys = o;   o += align16(kMpPiece * 4);
+  s.ml = o;     o += align16(G * 2 * 4);
+  s.misc = o;   o += align16(64 * 4);
+  o = (o + 127) & ~127;
+  s.region = o;
+  // scan: per-warp rings of centroid rows (the chunk top-k scratch reuses warp 0's ring)
+  s.ring = 0;
+  const int scan = kMpWarps * kMpScanSlots * kMpScanRows * kMpD * 4;
+  // merge of the request's candidates: keys, logical pages, page ids, top-k scratch
+  const int merge_small = 3 * 2 * kMpThreads * 4 + SmallTopk<kMpThreads>::BYTES;
+  const int merge_big = align16(g.cmax * 4) + align16(g.cmax * 2) + align16((kTopkBins + 64) * 4);
+  const int merge = merge_small > merge_big ? merge_small : merge_big;
+  // attention: the piece's K tiles (first: the merge scratch above is dead once they load),
+  // Q (prefetched while the merge runs), P, per-page maxima and sums
+  const int T = kMpPiece * kPage;
+  int a = 0;
+  s.kt = a; a += align16(T * kMpRow * 2);
+  s.q = a;  a += align16(G * kMpRow * 2);
+  s.pm = a; a += align16(G * (T + 8) * 2);
+  s.pmax = a; a += align16(kMpPiece * G * 4);
+  s.psum = a; a += align16(kMpPiece * G * 4);
+  int r = scan;
+  if (merge > r) r = merge;
+  if (a > r) r = a;
+  s.total = o + r;
+  return s;
+}
+
+
+__device__ __forceinline__ int mp_ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait (thread 0) until *ctr >= target; false (and VT_DEV_TIMEOUT) if it gave up.
+__device__ __forceinline__ bool mp_wait_at_least(const int32_t* ctr, int target, int32_t* status) {
+  if (mp_ld_acquire(ctr) >= target) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    __nanosleep(128);
+    if (mp_ld_acquire(ctr) >= target) return true;
+    if (global_ns() - t0 > kWaitNs) {
+      flag(status, kDevTimeout);
+      return false;
+    }
+  }
+}
+
+template <int G>
+__global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const DecodeParams p,
+                                                                    const MpWs w) {
+  constexpr int NT = kMpThreads;
+  constexpr int NW = kMpWarps;
+  constexpr int D = kMpD;
+  constexpr int DV = kMpDv;
+  constexpr int CH4 = D / 4;  // float4 per centroid row
+  constexpr int RB = D * 4;   // bytes of a centroid row
+  constexpr int T = kMpPiece * kPage;
+  constexpr int PST = T + 8;
+  static_assert(G == 16 || G == 32, "MLA path covers 16 or 32 query heads");
+  static_assert(kMpPiece >= 2, "the page-max table [kMpPiece][G] holds the merge's [G][2]");
+  static_assert(SmallTopk<NT>::BYTES <= kMpScanSlots * kMpScanRows * RB,
+                "the chunk top-k scratch fits in warp 0's ring");
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  const MpGeom gm = w.g;
+  const MpSmem Ls = mp_smem_layout(G, p.B, gm);
+  int* s_prefix = reinterpret_cast<int*>(smem + Ls.prefix);
+  uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem + Ls.keys);
+  int* s_pids = reinterpret_cast<int*>(smem + Ls.pids);
+  float* s_qm = reinterpret_cast<float*>(smem + Ls.qm);
+  int* s_sel = reinterpret_cast<int*>(smem + Ls.sel);
+  int* s_phys = reinterpret_cast<int*>(smem + Ls.phys);
+  float* s_ml = reinterpret_cast<float*>(smem + Ls.ml);
+  int* s_misc = reinterpret_cast<int*>(smem + Ls.misc);  // [0] item, [1] flag, [8..] scratch
+  unsigned char* region = smem + Ls.region;
+  const uint32_t region_u32 = smem_u32(region);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // programmatic dependent launch: nothing global is touched before the previous kernel ends
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+
+  uint32_t qbase = 0;  // thread 0: the claim count when this launch began
+  auto claim = [&]() { return (int)(atomicAdd(w.ctr + 0, 1u) - qbase); };
+
+  // ---- schedule: exclusive prefix of scan items over the requests
+  {
+    int first = 0;
+    if (tid == 0) {
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(qbase) : "l"(w.ctr + 1) : "memory");
+      first = claim();
+    }
+    const int per = (p.B + NT - 1) / NT;
+    const int i0 = min(p.B, tid * per), i1 = min(p.B, i0 + per);
+    int run = 0;
+    for (int i = i0; i < i1; ++i) {
+      const int c = mp_chunks(p.seq_lens[i], p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
+      s_prefix[i] = c;
+      run += c;
+    }
+    int x = run;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_misc[8 + warp] = x;
+    __syncthreads();
+    int base = 0;
+    for (int k = 0; k < warp; ++k) base += s_misc[8 + k];
+    int acc = base + x - run;
+    for (int i = i0; i < i1; ++i) {
+      const int c = s_prefix[i];
+      s_prefix[i] = acc;
+      acc += c;
+    }
+    if (tid == NT - 1) s_prefix[p.B] = base + x;
+    if (tid == 0) s_misc[0] = first;
+    __syncthreads();
+  }
+  // Queue order: block b holds the scan chunks of request b followed by the attention pieces
+  // of request b - lag, and the pieces of the last lag requests come at the end.  The
+  // attention (tensor-core bound here) then overlaps the scans (HBM bound) of later requests,
+  // and a request's chunks are about one round of CTAs ahead of its pieces.  Every wait
+  // is still for items earlier in the queue.
+  const int scan_items = s_prefix[p.B];
+  const int A = gm.A;
+  const int avg = (scan_items + p.B - 1) / p.B;
+  const int lag = min(p.B, (int)gridDim.x / (avg + A) + 1);
+  const int total_items = scan_items + p.B * A;
+  auto block_start = [&](int b) { return s_prefix[b] + A * max(0, b - lag); };
+
+  int32_t* pending = nullptr;  // thread 0: a counter to bump after the item's closing barrier
+  for (;;) {
+    const int t = s_misc[0];
+    __syncthreads();
+    if (t >= total_items) {
+      if (tid == 0 && t == total_items + (int)gridDim.x - 1)
+        w.ctr[1] = qbase + (uint32_t)total_items + gridDim.x;
+      break;
+    }
+    int next = -1;
+
+    // decode the item: (scan, request, chunk) or (attention, request, piece)
+    bool is_scan = false;
+    int ib, ic;
+    if (t >= block_start(p.B)) {
+      const int r = t - block_start(p.B);
+      ib = (p.B - lag) + r / A;
+      ic = r % A;
+    } else {
+      int lo = 0, hi = p.B - 1;  // the block holding t
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (block_start(mid) <= t) lo = mid; else hi = mid - 1;
+      }
+      const int r = t - block_start(lo), nc = s_prefix[lo + 1] - s_prefix[lo];
+      is_scan = r < nc;
+      ib = is_scan ? lo : lo - lag;
+      ic = is_scan ? r : r - nc;
+    }
+    if (is_scan) {
+      // ---------------------------------------------------------------- scan item
+      const int b = ib, c = ic;
+      const int L = p.seq_lens[b];
+      const int n = (L + kPage - 1) / kPage;
+      const int m = n - p.bos - p.eos;
+      const int c0 = c * kMlaChunk, cnt = min(kMlaChunk, m - c0);
+      const int32_t* ptrow = p.page_table + (int64_t)b * p.pt_stride;
+      // warp w: rows w + NW i (i < 16) of the chunk; lane i < 16 holds the page id of row i
+      const int myrows = (cnt - warp + NW - 1) / NW;
+      int pid = -1;
+      if (lane < myrows) {
+        pid = ptrow[p.bos + c0 + warp + NW * lane];
+        if (pid < 0 || pid >= p.num_pages) {
+          flag(p.status, VT_DEV_BAD_PAGE);
+          pid = -1;
+        }
+        s_pids[warp + NW * lane] = pid;
+      }
+      // fp32 mean of the request's G query heads: three groups of 72 threads each load every
+      // third row (one round of independent 16-byte loads), then sum through shared memory
+      const __nv_bfloat16* qb = p.q + (int64_t)b * p.Hq * D;
+      {
+        constexpr int NC8 = D / 8;  // 16-byte chunks per query row
+        float* s_part = reinterpret_cast<float*>(region);  // [3][D], in warp 0..2's rings, before use
+        const int grp = tid / NC8, c8 = tid - grp * NC8;
+        if (grp < 3) {
+          float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          constexpr int RPG = (G + 2) / 3;
+          uint4 raw[RPG];
+#pragma unroll
+          for (int k = 0; k < RPG; ++k) {
+            const int j = grp + 3 * k;
+            raw[k] = j < G ? *reinterpret_cast<const uint4*>(qb + (int64_t)j * D + c8 * 8)
+                           : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < RPG; ++k) {
+            a8[0] += bf_lo(raw[k].x); a8[1] += bf_hi(raw[k].x);
+            a8[2] += bf_lo(raw[k].y); a8[3] += bf_hi(raw[k].y);
+            a8[4] += bf_lo(raw[k].z); a8[5] += bf_hi(raw[k].z);
+            a8[6] += bf_lo(raw[k].w); a8[7] += bf_hi(raw[k].w);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) s_part[grp * D + c8 * 8 + e] = a8[e];
+        }
+        __syncthreads();
+        for (int d = tid; d < D; d += NT)
+          s_qm[d] = ((s_part[d] + s_part[D + d]) + s_part[2 * D + d]) / (float)G;
+      }
+      __syncthreads();  // the group mean is in shared memory
+      float4 qv[5];
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
+        const int cc = lane + 32 * i;
+        qv[i] = cc < CH4 ? reinterpret_cast<const float4*>(s_qm)[cc] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      const uint32_t ring = region_u32 + warp * kMpScanSlots * kMpScanRows * RB;
+      const int nb = (myrows + kMpScanRows - 1) / kMpScanRows;
+      auto issue = [&](int bt) {
+        if (bt < nb) {
+          const uint32_t dst = ring + (bt % kMpScanSlots) * kMpScanRows * RB;
+#pragma unroll
+          for (int rr = 0; rr < kMpScanRows; ++rr) {
+            const int i = bt * kMpScanRows + rr;  // uniform, < 16
+            const int pg = __shfl_sync(kFull, pid, i & 31);
+            if (i < myrows && pg >= 0) {
+              const float* crow = p.centroids + (int64_t)pg * D;
+              for (int cc = lane; cc < CH4; cc += 32) cp_async16(dst + rr * RB + cc * 16, crow + cc * 4, 16);
+            }
+          }
+        }
+        cp_async_commit();
+      };
+      uint32_t klo = 0xffffffffu, khi = 0u;
+#pragma unroll
+      for (int bt = 0; bt < kMpScanSlots - 1; ++bt) issue(bt);
+      for (int bt = 0; bt < nb; ++bt) {
+        issue(bt + kMpScanSlots - 1);
+        cp_async_wait<kMpScanSlots - 1>();
+        __syncwarp();
+        const uint32_t src = ring + (bt % kMpScanSlots) * kMpScanRows * RB;
+#pragma unroll
+        for (int rr = 0; rr < kMpScanRows; ++rr) {
+          float d = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 5; ++i) {
+            const int cc = lane + 32 * i;
+            if (cc < CH4) {
+              float4 cv;
+              asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+                           : "=f"(cv.x), "=f"(cv.y), "=f"(cv.z), "=f"(cv.w)
+                           : "r"(src + rr * RB + cc * 16));
+              d = fmaf(cv.x, qv[i].x, d);
+              d = fmaf(cv.y, qv[i].y, d);
+              d = fmaf(cv.z, qv[i].z, d);
+              d = fmaf(cv.w, qv[i].w, d);
+            }
+          }
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) d += __shfl_xor_sync(kFull, d, o);
+          const int i = bt * kMpScanRows + rr;
+          const int pg = __shfl_sync(kFull, pid, i & 31);
+          if (lane == 0 && i < myrows) {
+            const uint32_t key = score_key(pg >= 0 ? d : -INFINITY);
+            s_keys[warp + NW * i] = key;
+            klo = min(klo, key);
+            khi = max(khi, key);
+          }
+        }
+        __syncwarp();  // every lane is done with the slot before it is refilled
+      }
+      cp_async_wait<0>();
+      if (tid == 0) next = claim();
+      if (lane == 0) {
+        s_misc[16 + warp] = (int)klo;
+        s_misc[16 + NW + warp] = (int)khi;
+      }
+      unsigned char* tk = region;  // warp 0's ring, which only warp 0 has used
+      if (warp == 0)
+        for (int i = lane; i < SmallTopk<NT>::HIST / 4; i += 32)
+          reinterpret_cast<int4*>(tk)[i] = make_int4(0, 0, 0, 0);
+      __syncthreads();  // every score of the chunk is in s_keys; the rings are free
+      klo = 0xffffffffu;
+      khi = 0u;
+#pragma unroll
+      for (int k = 0; k < NW; ++k) {
+        klo = min(klo, (uint32_t)s_misc[16 + k]);
+        khi = max(khi, (uint32_t)s_misc[16 + NW + k]);
+      }
+      const int kc = min(gm.kc, cnt);
+      const int64_t cb = ((int64_t)b * gm.nch_max + c) * gm.kc;
+      uint32_t* ck = w.ckey + cb;
+      uint16_t* co = w.coff + cb;
+      int32_t* cp = w.cpid + cb;
+      small_topk<NT>(s_keys, cnt, kc, klo, khi, tk, [&](int j, int pos) {
+        ck[pos] = s_keys[j];
+        co[pos] = (uint16_t)j;
+        cp[pos] = s_pids[j];
+      });
+      pending = w.unit_done + b;
+    } else {
+      // ---------------------------------------------------------------- attention item
+      const int b = ib, piece = ic;
+      const int Ab = A, ppb = gm.pp;
+      const int L = p.seq_lens[b];
+      const int n = (L + kPage - 1) / kPage;
+      const bool valid = L >= 1 && n <= p.pt_stride;
+      const bool dense = n <= p.kmax;
+      const int nch = mp_chunks(L, p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
+      const int ns = !valid ? 0 : (dense ? n : p.kmax);
+      const int j0 = piece * ppb;
+      const int np = max(0, min(ns - j0, ppb));
+      const bool write_sel = piece == 0 && p.sel != nullptr;
+      int32_t* selrow = write_sel ? p.sel + (int64_t)b * p.kmax : nullptr;
+      const int64_t orow = (int64_t)b * p.Hq;
+      const int32_t* ptrow = p.page_table + (int64_t)b * p.pt_stride;
+      if (tid == 0 && piece == 0) {
+        if (!valid) flag(p.status, VT_DEV_BAD_LEN);
+        if (p.n_sel) p.n_sel[b] = ns;
+      }
+      // Q (G x 576) for the attention below, fetched while the wait and the merge run (its slot
+      // lies past every merge scratch of the small path)
+      const int m_c = n - p.bos - p.eos;
+      const int C_c = nch > 0 ? (nch - 1) * gm.kc + min(gm.kc, m_c - (nch - 1) * kMlaChunk) : 0;
+      const bool q_early = C_c <= 2 * NT;
+      __nv_bfloat16* s_q = reinterpret_cast<__nv_bfloat16*>(region + Ls.q);
+      auto stage_q = [&]() {
+        for (int i = tid; i < G * (D / 8); i += NT) {
+          const int g = i / (D / 8), c8 = i - g * (D / 8);
+          cp_async16(smem_u32(s_q + g * kMpRow + c8 * 8), p.q + (orow + g) * D + c8 * 8, 16);
+        }
+        cp_async_commit();
+      };
+      if (q_early) stage_q();
+      int ok = 1;
+      if (nch > 0) {  // every chunk of the request has stored its candidates
+        if (tid == 0) s_misc[1] = mp_wait_at_least(w.unit_done + b, nch, p.status) ? 1 : 0;
+        __syncthreads();
+        ok = s_misc[1];
+      }
+      if (ok) {
+        // ---- the logical pages of this piece into s_sel[0, np), their page ids into s_phys
+        auto phys_of = [&](int lp) {
+          int pg = ptrow[lp];
+          if (pg < 0 || pg >= p.num_pages) {
+            flag(p.status, VT_DEV_BAD_PAGE);
+            pg = -1;
+          }
+          return pg;
+        };
+        bool have_phys = false;
+        if (nch > 0) {
+          const int m = n - p.bos - p.eos;
+          const int kc = gm.kc;
+          const int C = (nch - 1) * kc + min(kc, m - (nch - 1) * kMlaChunk);
+          const int64_t cb = (int64_t)b * gm.nch_max * kc;  // chunks are contiguous
+          const int bos = p.bos, topk = p.topk;
+          for (int q = tid; q < np; q += NT) {  // reserved pages of the piece
+            const int pos = j0 + q;
+            if (pos < bos || pos >= bos + topk) {
+              const int lp = pos < bos ? pos : n - p.eos + (pos - bos - topk);
+              s_sel[q] = lp;
+              s_phys[q] = phys_of(lp);
+            }
+          }
+          if (write_sel) {
+            for (int j = tid; j < bos; j += NT) selrow[j] = j;
+            for (int j = tid; j < p.eos; j += NT) selrow[bos + topk + j] = n - p.eos + j;
+          }
+          // candidate j of chunk j / kc sits at offset coff[j] of it; candidates are in
+          // ascending page order, so ties (lowest position) go to the lowest page
+          if (C <= 2 * NT) {
+            uint32_t* keys = reinterpret_cast<uint32_t*>(region);
+            int* lps = reinterpret_cast<int*>(region + 2 * NT * 4);
+            int* pids = reinterpret_cast<int*>(region + 4 * NT * 4);
+            unsigned char* tk = region + 6 * NT * 4;
+            for (int i = tid; i < SmallTopk<NT>::HIST / 4; i += NT)
+              reinterpret_cast<int4*>(tk)[i] = make_int4(0, 0, 0, 0);
+            uint32_t klo = 0xffffffffu, khi = 0u;
+            for (int j = tid; j < C; j += NT) {
+              const uint32_t key = __ldcg(w.ckey + cb + j);
+              keys[j] = key;
+              lps[j] = bos + (j / kc) * kMlaChunk + __ldcg(w.coff + cb + j);
+              pids[j] = __ldcg(w.cpid + cb + j);
+              klo = min(klo, key);
+              khi = max(khi, key);
+            }
+            klo = __reduce_min_sync(kFull, klo);
+            khi = __reduce_max_sync(kFull, khi);
+            if (lane == 0) {
+              s_misc[16 + warp] = (int)klo;
+              s_misc[16 + NW + warp] = (int)khi;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int k = 0; k < NW; ++k) {
+              klo = min(klo, (uint32_t)s_misc[16 + k]);
+              khi = max(khi, (uint32_t)s_misc[16 + NW + k]);
+            }
+            small_topk<NT>(keys, C, topk, klo, khi, tk, [&](int j, int pos) {
+              const int q = bos + pos - j0;
+              if (q >= 0 && q < np) {
+                s_sel[q] = lps[j];
+                int pg = pids[j];
+                if (pg < 0 || pg >= p.num_pages) {
+                  flag(p.status, VT_DEV_BAD_PAGE);
+                  pg = -1;
+                }
+                s_phys[q] = pg;
+              }
+              if (write_sel) selrow[bos + pos] = lps[j];
+            });
+            have_phys = true;
+          } else {
+            uint32_t* keys = reinterpret_cast<uint32_t*>(region);
+            uint16_t* offs = reinterpret_cast<uint16_t*>(region + align16(gm.cmax * 4));
+            int* hist = reinterpret_cast<int*>(region + align16(gm.cmax * 4) + align16(gm.cmax * 2));
+            for (int j = tid; j < C; j += NT) {
+              keys[j] = __ldcg(w.ckey + cb + j);
+              offs[j] = __ldcg(w.coff + cb + j);
+            }
+            __syncthreads();
+            block_topk<NT>(keys, C, topk, hist, hist + kTopkBins, [&](int j, int pos) {
+              const int lp = bos + (j / kc) * kMlaChunk + offs[j];
+              const int q = bos + pos - j0;
+              if (q >= 0 && q < np) s_sel[q] = lp;
+              if (write_sel) selrow[bos + pos] = lp;
+            });
+          }
+        } else {
+          // dense (every page, in order) or, with topk == 0, the reserved pages alone
+          const bool resv = valid && !dense;
+          auto page_at = [&](int pos) {
+            return (!resv || pos < p.bos) ? pos : n - p.eos + (pos - p.bos);
+          };
+          for (int q = tid; q < np; q += NT) s_sel[q] = page_at(j0 + q);
+          if (write_sel)
+            for (int j = tid; j < p.kmax; j += NT) selrow[j] = j < ns ? page_at(j) : -1;
+        }
+        __syncthreads();
+        if (!have_phys) {
+          if (tid < np) s_phys[tid] = phys_of(s_sel[tid]);
+          __syncthreads();
+        }
+        // ---- stage the piece's K tiles (zero rows past the valid tokens), and Q if not yet
+        __nv_bfloat16* s_kt = reinterpret_cast<__nv_bfloat16*>(region + Ls.kt);
+        __nv_bfloat16* s_pm = reinterpret_cast<__nv_bfloat16*>(region + Ls.pm);  // [G][T+8]
+        float* s_pmax = reinterpret_cast<float*>(region + Ls.pmax);             // [piece page][G]
+        float* s_psum = reinterpret_cast<float*>(region + Ls.psum);             // [piece page][G]
+        const int last_valid = L - kPage * (n - 1);
+        if (!q_early) stage_q();
+        // warp w loads page w of the piece itself, so that its S^T can start as soon as its
+        // own tile has landed (every thread commits the group, empty or not)
+        if (warp < np) {
+          const int pg = s_phys[warp];
+          const bool lastp = s_sel[warp] == n - 1;
+          for (int i = lane; i < kPage * (D / 8); i += 32) {
+            const int tt = i / (D / 8), c8 = i - tt * (D / 8);
+            const bool ok_row = pg >= 0 && (!lastp || tt < last_valid);
+            const __nv_bfloat16* src =
+                ok_row ? p.k_pool + (int64_t)pg * p.sk_p + (int64_t)tt * p.sk_t + c8 * 8 : p.k_pool;
+            cp_async16(smem_u32(s_kt + (warp * 16 + tt) * kMpRow + c8 * 8), src, ok_row ? 16 : 0);
+          }
+        }
+        cp_async_commit();
+        cp_async_wait<1>();  // this thread's share of Q has landed
+        __syncthreads();     // all of Q has
+        cp_async_wait<0>();  // and this warp's page
+        __syncwarp();
+        // ---- S^T = K Q^T: warp w owns page w (16 tokens) x all G heads, kept in registers:
+        // this lane holds tokens r0 = lane/4 and r0 + 8, heads nt*8 + 2 (lane%4) + {0, 1}
+        float acc[G / 8][4];
+#pragma unroll
+        for (int nt = 0; nt < G / 8; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+        if (warp < np) {
+          const uint32_t a_base = smem_u32(s_kt + (warp * 16 + (lane & 15)) * kMpRow + (lane >> 4) * 8);
+          const uint32_t b_base =
+              smem_u32(s_q + ((lane & 7) + ((lane >> 4) << 3)) * kMpRow + ((lane >> 3) & 1) * 8);
+#pragma unroll 4
+          for (int ks = 0; ks < D / 16; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(a_base + ks * 32, a0, a1, a2, a3);
+#pragma unroll
+            for (int n2 = 0; n2 < G / 16; ++n2) {
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4(b_base + n2 * 16 * kMpRow * 2 + ks * 32, b0, b1, b2, b3);
+              mma_16816(acc[2 * n2], a0, a1, a2, a3, b0, b1);
+              mma_16816(acc[2 * n2 + 1], a0, a1, a2, a3, b2, b3);
+            }
+          }
+        }
+        // ---- softmax over the piece's tokens, per head: page maxima, then probabilities
+        // against the piece's maximum (rounded once to bf16, as the P V MMA reads them)
+        const int r0 = lane >> 2;
+        bool v0 = false, v1 = false;
+        if (warp < np) {
+          const bool live = s_phys[warp] >= 0, lastp = s_sel[warp] == n - 1;
+          v0 = live && (!lastp || r0 < last_valid);
+          v1 = live && (!lastp || r0 + 8 < last_valid);
+        }
+#pragma unroll
+        for (int nt = 0; nt < G / 8; ++nt) {
+          acc[nt][0] = v0 ? acc[nt][0] * p.qscale : -INFINITY;
+          acc[nt][1] = v0 ? acc[nt][1] * p.qscale : -INFINITY;
+          acc[nt][2] = v1 ? acc[nt][2] * p.qscale : -INFINITY;
+          acc[nt][3] = v1 ? acc[nt][3] * p.qscale : -INFINITY;
+          float m0 = fmaxf(acc[nt][0], acc[nt][2]), m1 = fmaxf(acc[nt][1], acc[nt][3]);
+#pragma unroll
+          for (int o = 4; o <= 16; o <<= 1) {
+            m0 = fmaxf(m0, __shfl_xor_sync(kFull, m0, o));
+            m1 = fmaxf(m1, __shfl_xor_sync(kFull, m1, o));
+          }
+          if (warp < np && lane < 4) {
+            s_pmax[warp * G + nt * 8 + 2 * lane] = m0;
+            s_pmax[warp * G + nt * 8 + 2 * lane + 1] = m1;
+          }
+        }
+        __syncthreads();
+        if (warp < np) {
+#pragma unroll
+          for (int nt = 0; nt < G / 8; ++nt) {
+            const int c = nt * 8 + 2 * (lane & 3);
+            float M0 = -INFINITY, M1 = -INFINITY;
+            for (int q = 0; q < np; ++q) {
+              M0 = fmaxf(M0, s_pmax[q * G + c]);
+              M1 = fmaxf(M1, s_pmax[q * G + c + 1]);
+            }
+            const __nv_bfloat16 p00 = __float2bfloat16(acc[nt][0] == -INFINITY ? 0.0f : exp2f(acc[nt][0] - M0));
+            const __nv_bfloat16 p01 = __float2bfloat16(acc[nt][1] == -INFINITY ? 0.0f : exp2f(acc[nt][1] - M1));
+            const __nv_bfloat16 p10 = __float2bfloat16(acc[nt][2] == -INFINITY ? 0.0f : exp2f(acc[nt][2] - M0));
+            const __nv_bfloat16 p11 = __float2bfloat16(acc[nt][3] == -INFINITY ? 0.0f : exp2f(acc[nt][3] - M1));
+            const int tk = warp * 16 + r0;
+            s_pm[c * PST + tk] = p00;
+            s_pm[(c + 1) * PST + tk] = p01;
+            s_pm[c * PST + tk + 8] = p10;
+            s_pm[(c + 1) * PST + tk + 8] = p11;
+            // the sums use the rounded weights, as the MMA does
+            float l0 = __bfloat162float(p00) + __bfloat162float(p10);
+            float l1 = __bfloat162float(p01) + __bfloat162float(p11);
+#pragma unroll
+            for (int o = 4; o <= 16; o <<= 1) {
+              l0 += __shfl_xor_sync(kFull, l0, o);
+              l1 += __shfl_xor_sync(kFull, l1, o);
+            }
+            if (lane < 4) {
+              s_psum[warp * G + c] = l0;
+              s_psum[warp * G + c + 1] = l1;
+            }
+          }
+        }
+        __syncthreads();
+        for (int g = tid; g < G; g += NT) {
+          float M = -INFINITY, Ls = 0.0f;
+          for (int q = 0; q < np; ++q) {
+            M = fmaxf(M, s_pmax[q * G + g]);
+            Ls += s_psum[q * G + g];
+          }
+          s_ml[2 * g] = M;
+          s_ml[2 * g + 1] = Ls;
+        }
+        __syncthreads();
+        // ---- O = P V: warp w owns output dims [64 w, 64 w + 64) for all G heads
+        float oacc[G / 16][8][4];
+#pragma unroll
+        for (int mt = 0; mt < G / 16; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) oacc[mt][nt][i] = 0.0f;
+        {
+          const uint32_t pa_base = smem_u32(s_pm + (lane & 15) * PST + (lane >> 4) * 8);
+          const uint32_t vb_base = smem_u32(s_kt + ((lane & 7) + ((lane >> 3) & 1) * 8) * kMpRow +
+                                            warp * 64 + (lane >> 4) * 8);
+          for (int ks = 0; ks < np; ++ks) {  // 16 tokens per step
+            uint32_t ar[G / 16][4];
+#pragma unroll
+            for (int mt = 0; mt < G / 16; ++mt)
+              ldsm_x4(pa_base + (mt * 16 * PST + ks * 16) * 2, ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3]);
+#pragma unroll
+            for (int n2 = 0; n2 < 4; ++n2) {
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4_t(vb_base + (ks * 16 * kMpRow + n2 * 16) * 2, b0, b1, b2, b3);
+#pragma unroll
+              for (int mt = 0; mt < G / 16; ++mt) {
+                mma_16816(oacc[mt][2 * n2], ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3], b0, b1);
+                mma_16816(oacc[mt][2 * n2 + 1], ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3], b2, b3);
+              }
+            }
+          }
+        }
+        // ---- finish: this lane holds heads g = 16 mt + lane/4 (+8), dims 64 warp + 8 nt + 2 (lane%4) (+1)
+        auto write_out = [&](float (&o)[G / 16][8][4], auto&& ml_of) {
+#pragma unroll
+          for (int mt = 0; mt < G / 16; ++mt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int g = mt * 16 + (lane >> 2) + 8 * hh;
+              const float2 ml = ml_of(g);
+              const float inv = ml.y > 0.0f ? 1.0f / ml.y : 0.0f;
+#pragma unroll
+              for (int nt = 0; nt < 8; ++nt) {
+                const int d = warp * 64 + nt * 8 + 2 * (lane & 3);
+                __nv_bfloat162 v2;
+                v2.x = __float2bfloat16(o[mt][nt][2 * hh] * inv);
+                v2.y = __float2bfloat16(o[mt][nt][2 * hh + 1] * inv);
+                *reinterpret_cast<__nv_bfloat162*>(p.out + (orow + g) * DV + d) = v2;
+              }
+              if (warp == 0 && (lane & 3) == 0 && p.lse)
+                p.lse[orow + g] = ml.y > 0.0f ? (ml.x + log2f(ml.y)) * kLn2 : -INFINITY;
+            }
+        };
+        if (Ab == 1) {
+          write_out(oacc, [&](int g) { return make_float2(s_ml[2 * g], s_ml[2 * g + 1]); });
+          if (tid == 0 && nch > 0) w.unit_done[b] = 0;
+        } else if (piece < Ab - 1) {
+          // publish this piece's partial and move on: the request's last piece merges them
+          float* dst = w.part + ((int64_t)b * A + piece) * G * (DV + 2);
+#pragma unroll
+          for (int mt = 0; mt < G / 16; ++mt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int g = mt * 16 + (lane >> 2) + 8 * hh;
+#pragma unroll
+              for (int nt = 0; nt < 8; ++nt) {
+                const int d = warp * 64 + nt * 8 + 2 * (lane & 3);
+                *reinterpret_cast<float2*>(dst + g * (DV + 2) + d) =
+                    make_float2(oacc[mt][nt][2 * hh], oacc[mt][nt][2 * hh + 1]);
+              }
+            }
+          for (int g = tid; g < G; g += NT)
+            *reinterpret_cast<float2*>(dst + g * (DV + 2) + DV) = make_float2(s_ml[2 * g], s_ml[2 * g + 1]);
+          pending = w.att_cnt + b;
+        } else {
+          // the last piece: wait for the other Ab - 1 partials (claimed before this item, and
+          // they never wait on a later one), then merge them into this piece's registers
+          if (tid == 0) s_misc[1] = mp_wait_at_least(w.att_cnt + b, Ab - 1, p.status) ? 1 : 0;
+          __syncthreads();
+          if (s_misc[1]) {
+            const float* src = w.part + (int64_t)b * A * G * (DV + 2);
+            // per head: the merged max and the rescaled sum (the page-max table is free again)
+            float* s_mm = s_pmax;  // [G][2]
+            for (int g = tid; g < G; g += NT) {
+              float M = s_ml[2 * g];
+              for (int q = 0; q < Ab - 1; ++q) M = fmaxf(M, __ldcg(src + (q * G + g) * (DV + 2) + DV));
+              float Lsum = (s_ml[2 * g] == -INFINITY) ? 0.0f : s_ml[2 * g + 1] * exp2f(s_ml[2 * g] - M);
+              for (int q = 0; q < Ab - 1; ++q) {
+                const float mq = __ldcg(src + (q * G + g) * (DV + 2) + DV);
+                if (mq != -INFINITY) Lsum = fmaf(__ldcg(src + (q * G + g) * (DV + 2) + DV + 1), exp2f(mq - M), Lsum);
+              }
+              s_mm[2 * g] = M;
+              s_mm[2 * g + 1] = Lsum;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int mt = 0; mt < G / 16; ++mt)
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const int g = mt * 16 + (lane >> 2) + 8 * hh;
+                const float M = s_mm[2 * g];
+                const float fo = (s_ml[2 * g] == -INFINITY) ? 0.0f : exp2f(s_ml[2 * g] - M);
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) {
+                  oacc[mt][nt][2 * hh] *= fo;
+                  oacc[mt][nt][2 * hh + 1] *= fo;
+                }
+                for (int q = 0; q < Ab - 1; ++q) {
+                  const float* pq = src + (q * G + g) * (DV + 2);
+                  const float mq = __ldcg(pq + DV);
+                  const float f = (mq == -INFINITY) ? 0.0f : exp2f(mq - M);
+#pragma unroll
+                  for (int nt = 0; nt < 8; ++nt) {
+                    const int d = warp * 64 + nt * 8 + 2 * (lane & 3);
+                    const float2 v = __ldcg(reinterpret_cast<const float2*>(pq + d));
+                    oacc[mt][nt][2 * hh] = fmaf(v.x, f, oacc[mt][nt][2 * hh]);
+                    oacc[mt][nt][2 * hh + 1] = fmaf(v.y, f, oacc[mt][nt][2 * hh + 1]);
+                  }
+                }
+              }
+            write_out(oacc, [&](int g) { return make_float2(s_mm[2 * g], s_mm[2 * g + 1]); });
+            if (tid == 0) {  // every piece is past its waits: reset the request's counters
+              w.att_cnt[b] = 0;
+              w.unit_done[b] = 0;
+            }
+          }
+        }
+      }
+    }
+    if (tid == 0) s_misc[0] = next >= 0 ? next : claim();
+    __syncthreads();
+    if (tid == 0 && pending != nullptr) {
+      // the barrier above ordered every thread's stores of the item before this fence
+      __threadfence();
+      atomicAdd(pending, 1);
+      pending = nullptr;
+    }
+  }
+}
+
+
+// ---- host side ----------------------------------------------------------------------------
+
+size_t mla_persist_workspace_bytes(const DecodeParams& p, int G, int64_t unit_cap) {
+  return mp_ws_layout(p, G, unit_cap).total;
+}
+
+int mla_persist_smem_bytes(const DecodeParams& p, int G) {
+  return mp_smem_layout(G, p.B, mp_geom(p.pt_stride, p.topk, p.bos, p.eos, p.kmax)).total;
+}
+
+int mla_persist_max_batch() { return kMpMaxB; }
+
+template <int G>
+static cudaError_t launch_mla_persist_t(const DecodeParams& p, const MpWs& w, int sm_count,
+                                        cudaStream_t stream) {
+  auto kern = persist_mla_kernel<G>;
+  const int smem = mp_smem_layout(G, p.B, w.g).total;
+  static std::atomic<int> optin[64];
+  cudaError_t e = ensure_smem_optin(kern, smem, false, optin);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kMpThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sm_count * per_sm);
+  cfg.blockDim = dim3(kMpThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p, w);
+}
+
+// The fused MLA call on `ws` (mla_persist_workspace_bytes() bytes for the same unit_cap,
+// counters zero): as many CTAs as fit on the sm_count SMs at once.
+cudaError_t launch_mla_persist(const DecodeParams& p, int G, void* ws, int64_t unit_cap,
+                               int sm_count, cudaStream_t s) {
+  const MpWsLayout L = mp_ws_layout(p, G, unit_cap);
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  MpWs w;
+  w.ctr = reinterpret_cast<uint32_t*>(base + L.ctr);
+  w.unit_done = reinterpret_cast<int32_t*>(base + L.unit_done);
+  w.att_cnt = reinterpret_cast<int32_t*>(base + L.att_cnt);
+  w.ckey = reinterpret_cast<uint32_t*>(base + L.ckey);
+  w.coff = reinterpret_cast<uint16_t*>(base + L.coff);
+  w.cpid = reinterpret_cast<int32_t*>(base + L.cpid);
+  w.part = reinterpret_cast<float*>(base + L.part);
+  w.g = mp_geom(p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
+  if (G == 16) return launch_mla_persist_t<16>(p, w, sm_count, s);
+  if (G == 32) return launch_mla_persist_t<32>(p, w, sm_count, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vt

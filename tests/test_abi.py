@@ -125,10 +125,12 @@ def test_fused_workspace_contract(lib):
     assert _fused(lib, kv, a, ws=None, ws_bytes=0) == INV                   # missing
     assert _fused(lib, kv, a, ws=FAKE, ws_bytes=need - 1) == INV            # too small
     assert _fused(lib, kv, a, ws=FAKE + 16, ws_bytes=need) == INV           # misaligned
-    # MLA and very large batches need none
+    # MLA takes its own persistent path (with a workspace); very large batches need none
     mla = _kv(num_kv_heads=1, head_dim=576, head_dim_v=512, v_pool=FAKE, sk_h=576, sv_h=576,
               sk_p=16 * 576, sv_p=16 * 576, sk_t=576, sv_t=576)
-    assert lib.vt_fused_workspace_size(ctypes.byref(mla), ctypes.byref(_args(num_q_heads=32))) == 0
+    assert lib.vt_fused_workspace_size(ctypes.byref(mla), ctypes.byref(_args(num_q_heads=32))) > 0
+    assert lib.vt_fused_workspace_size(ctypes.byref(mla),
+                                       ctypes.byref(_args(num_q_heads=32, batch=5000))) == 0
     assert lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(_args(batch=5000))) == 0
     assert lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(_args(topk=-1))) == 0
     # grows with the batch and with the chunks of the page-table row
