@@ -30,6 +30,14 @@ CASES = {
     "g7_d64": dict(cfg=1, B=3, Hq=7, Hkv=1, len_lo=300, len_hi=2000, pool_pages=500, lengths="uniform"),
     "g8_d128": dict(cfg=2, B=3, Hq=16, Hkv=2, len_lo=700, len_hi=3000, pool_pages=800),
     "mla16": dict(cfg=4, B=2, Hq=16, len_lo=2500, len_hi=2500, pool_pages=400),
+    # top-k large enough that the chunks keep more candidates than the fused merge's fast path
+    # takes (GQA: more than 256; MLA: more than 512, and 13 attention pieces per request)
+    "bigk_gqa": dict(cfg=2, B=3, Hq=4, Hkv=2, topk=300, len_lo=18000, len_hi=22000,
+                     pool_pages=5000),
+    "bigk_mla": dict(cfg=4, B=2, Hq=16, topk=100, len_lo=16000, len_hi=16000, pool_pages=2100),
+    # more requests than the persistent path takes: the fused call runs the cluster kernel
+    "big_batch": dict(cfg=1, B=2100, len_lo=200, len_hi=900, lengths="uniform",
+                      pool_pages=80000),
 }
 
 
