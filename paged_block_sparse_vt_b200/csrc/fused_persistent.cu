@@ -11,7 +11,7 @@
 // sparse-attention speedups are lost).
 //
 // Work items, claimed in order through one global counter (a CTA claims its next item when
-// the streaming part of the current one is done, so the counter's latency is hidden by the
+// the streaming part of the current one is ending, so the counter's latency is hidden by the
 // current item's tail and the queue order still follows the CTAs' actual progress):
 //   scan items   -- (request, KV head, chunk of kChunk candidate pages), in request order,
 //                   each unit's chunks consecutive.  Every warp streams its rows of the
@@ -19,6 +19,8 @@
 //                   fp32 mean of the unit's G query heads; the CTA then takes the exact top-k
 //                   of the chunk in shared memory and stores those candidates (ordered
 //                   score key and offset, ascending by page) before counting the chunk done.
+//                   When the next item is a scan item too, its page ids and first batches
+//                   are put in flight before that top-k, so the CTA's loads do not pause.
 //                   The union of the chunks' top-k holds the unit's top-k: a key outside its
 //                   chunk's top-k has k keys above it in that chunk alone;
 //   attention    -- (unit, piece of at most kPiecePages selected pages), after every scan item.  The
@@ -26,8 +28,8 @@
 //                   claimed before this item and scan items never wait, so the wait ends),
 //                   merges the candidates with the same exact top-k, attends the pages of its
 //                   piece on the tensor cores (four per warp through a two-slot ring) and
-//                   stores a partial (max, sum, acc); the CTA that completes a unit's last
-//                   piece merges the partials and writes the bf16 output and the lse.
+//                   stores a partial (max, sum, acc); the piece that is counted last for
+//                   its unit merges the partials and writes the bf16 output and the lse.
 // The schedule (scan items per request and their prefix) is computed by every CTA from the
 // sequence lengths at start, so the call is one launch.  The per-unit counters are reset by
 // the CTA that last uses them and the claim counter runs on across launches (each launch
@@ -129,6 +131,16 @@ static PersistWsLayout persist_ws_layout(const DecodeParams& p, int G, int Dv, i
 
 // ---- memory-order helpers (gpu scope) --------------------------------------------------
 
+__device__ __forceinline__ void red_release_add(int32_t* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int atom_acq_rel_add(int32_t* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
@@ -165,7 +177,9 @@ __host__ __device__ inline PersistSmem persist_smem_layout(int D, int G, int B,
   s.misc = o;   o += align16(64 * 4);
   o = (o + 127) & ~127;
   s.region = o;  // one of: scan rings | top-k scratch | page rings | attention partials
-  const int scan = kPersistWarps * kScanRing * 8 * D * 4;
+  // scan rings, plus the chunk top-k scratch where it does not fit in one ring slot
+  const int scan = kPersistWarps * kScanRing * 8 * D * 4 +
+                   (8 * D * 4 >= SmallTopk<kPersistThreads>::BYTES ? 0 : SmallTopk<kPersistThreads>::BYTES);
   const int att = kPersistWarps * 2 * 2 * kPage * (D + 8) * 2;
   // merge of up to 2 NT candidates: keys, logical and physical pages, small_topk scratch;
   // of more: keys, offsets, block_topk scratch
@@ -192,8 +206,7 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
   constexpr int RPS = 32 / LPR_S;  // centroid rows per warp step
   constexpr int SN = 8 / RPS;      // values per lane per batch of 8 rows
   static_assert(D == 64 || D == 128, "GQA path covers head_dim 64 and 128");
-  static_assert(SmallTopk<kPersistThreads>::BYTES <= kScanRing * 8 * D * 4,
-                "the chunk top-k scratch fits in warp 0's scan ring");
+  static_assert(kPiecePages <= kPersistThreads, "one thread per page of a piece");
 
   extern __shared__ __align__(128) unsigned char smem[];
   const PersistGeom gm = w.g;
@@ -260,8 +273,86 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
   const int total_items = scan_items + u_split * gm.A + (w.units - u_split) * gm.A2;
 
   // A counter that thread 0 bumps (release) once the CTA has passed the barrier at the end
-  // of the item that produced the counted data, so that the fence overlaps the next item.
+  // of the item that produced the counted data.
   int32_t* pending = nullptr;
+
+  // ---- scan items: where an item's rows lie, and its per-lane state.  A scan item whose
+  // predecessor was a scan item finds its page ids and query mean already in registers and
+  // its first kScanRing - 1 batches in flight (prepared during the predecessor's top-k).
+  struct ScanItem {
+    int b, h, c, u, cnt, c0, myrows, batches;
+  };
+  auto scan_item = [&](int t) {
+    ScanItem it;
+    int lo = 0, hi = p.B - 1;  // largest k with prefix[k] <= t: a request with items
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_prefix[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    it.b = lo;
+    const int r = t - s_prefix[it.b];
+    const int n = (p.seq_lens[it.b] + kPage - 1) / kPage;
+    const int m = n - p.bos - p.eos;
+    const int nch = (m + kChunk - 1) / kChunk;
+    it.h = r / nch;
+    it.c = r - it.h * nch;
+    it.u = it.b * p.Hkv + it.h;
+    it.c0 = it.c * kChunk;
+    it.cnt = min(kChunk, m - it.c0);
+    // warp w: rows w + NW i, i < 64 of the chunk, streamed in batches of 8
+    it.myrows = (it.cnt - warp + NW - 1) / NW;
+    it.batches = (it.myrows + 7) / 8;
+    return it;
+  };
+  const int sub = lane / LPR_S, ch = lane % LPR_S;
+  bool prepared = false;
+  int pidA = -1, pidB = -1;  // lane l: page ids of its warp's rows l and l + 32
+  float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);  // fp32 group mean of q, this lane's float4
+  auto scan_fetch = [&](const ScanItem& it) {
+    const __nv_bfloat16* q0 = p.q + ((int64_t)it.b * p.Hq + (int64_t)it.h * G) * D + ch * 4;
+    const int32_t* ptrow = p.page_table + (int64_t)it.b * p.pt_stride + p.bos + it.c0 + warp;
+    pidA = lane < it.myrows ? ptrow[NW * lane] : -1;
+    pidB = lane + 32 < it.myrows ? ptrow[NW * (lane + 32)] : -1;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      const uint2 raw = *reinterpret_cast<const uint2*>(q0 + (int64_t)j * D);
+      a.x += bf_lo(raw.x);
+      a.y += bf_hi(raw.x);
+      a.z += bf_lo(raw.y);
+      a.w += bf_hi(raw.y);
+    }
+    qv = make_float4(a.x / (float)G, a.y / (float)G, a.z / (float)G, a.w / (float)G);
+    if (pidA >= p.num_pages || pidA < -1 || pidB >= p.num_pages || pidB < -1 ||
+        (lane < it.myrows && pidA < 0) || (lane + 32 < it.myrows && pidB < 0)) {
+      flag(p.status, VT_DEV_BAD_PAGE);
+      if (pidA < 0 || pidA >= p.num_pages) pidA = -1;
+      if (pidB < 0 || pidB >= p.num_pages) pidB = -1;
+    }
+  };
+  constexpr int CPRS = S::C_ROW / 16;  // 16-byte chunks per centroid row
+  const int64_t cstride = (int64_t)p.Hkv * D;
+  auto scan_issue = [&](const ScanItem& it, int bt) {
+    if (bt < it.batches) {
+      const uint32_t dst = region_u32 + (warp * kScanRing + bt % kScanRing) * 8 * S::C_ROW;
+      const float* cbase = p.centroids + (int64_t)it.h * D;
+#pragma unroll
+      for (int t8 = 0; t8 < 8; ++t8) {
+        const int i = bt * 8 + t8;  // uniform, < 64
+        const int pg = __shfl_sync(kFull, i < 32 ? pidA : pidB, i & 31);
+#pragma unroll
+        for (int kk = lane; kk < CPRS; kk += 32)
+          if (pg >= 0)
+            cp_async16(dst + t8 * S::C_ROW + kk * 16, cbase + (int64_t)pg * cstride + kk * 4, 16);
+      }
+    }
+    cp_async_commit();
+  };
+  // scratch of a chunk's top-k: warp 0's last ring slot where it is large enough (the next
+  // item's first batches fill the other slots meanwhile), else past the rings
+  unsigned char* tk = region + (8 * S::C_ROW >= SmallTopk<NT>::BYTES
+                                    ? (kScanRing - 1) * 8 * S::C_ROW
+                                    : NW * kScanRing * 8 * S::C_ROW);
   for (;;) {
     const int t = s_misc[0];
     __syncthreads();  // every thread has read the item before the next claim is stored
@@ -278,76 +369,23 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
 
     if (t < scan_items) {
       // ---------------------------------------------------------------- scan item
-      int lo = 0, hi = p.B - 1;  // largest k with prefix[k] <= t: a request with items
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_prefix[mid] <= t) lo = mid; else hi = mid - 1;
-      }
-      const int b = lo;
-      const int r = t - s_prefix[b];
-      const int L = p.seq_lens[b];
-      const int n = (L + kPage - 1) / kPage;
-      const int m = n - p.bos - p.eos;
-      const int nch = (m + kChunk - 1) / kChunk;
-      const int h = r / nch, c = r - h * nch;
-      const int u = b * p.Hkv + h;
-      const int32_t* ptrow = p.page_table + (int64_t)b * p.pt_stride;
-      const int c0 = c * kChunk;
-      const int cnt = min(kChunk, m - c0);
-      // fp32 mean of the group's queries for this lane's float4 of the row
-      const int sub = lane / LPR_S, ch = lane % LPR_S;
-      float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
-      {
-        const __nv_bfloat16* q0 = p.q + ((int64_t)b * p.Hq + (int64_t)h * G) * D + ch * 4;
+      const ScanItem it = scan_item(t);
+      if (!prepared) {
+        scan_fetch(it);
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-          const uint2 raw = *reinterpret_cast<const uint2*>(q0 + (int64_t)j * D);
-          qv.x += bf_lo(raw.x);
-          qv.y += bf_hi(raw.x);
-          qv.z += bf_lo(raw.y);
-          qv.w += bf_hi(raw.y);
-        }
-        qv.x /= (float)G; qv.y /= (float)G; qv.z /= (float)G; qv.w /= (float)G;
+        for (int bt = 0; bt < kScanRing - 1; ++bt) scan_issue(it, bt);
       }
-      // warp w: rows w + NW i, i < 64 of the chunk; lane l holds the page ids of rows l and
-      // l + 32, then streams the rows in batches of 8 through its kScanRing-slot ring
-      const int myrows = (cnt - warp + NW - 1) / NW;
-      int pidA = -1, pidB = -1;
-      if (lane < myrows) pidA = ptrow[p.bos + c0 + warp + NW * lane];
-      if (lane + 32 < myrows) pidB = ptrow[p.bos + c0 + warp + NW * (lane + 32)];
-      if (pidA >= p.num_pages || pidA < -1 || pidB >= p.num_pages || pidB < -1 ||
-          (lane < myrows && pidA < 0) || (lane + 32 < myrows && pidB < 0)) {
-        flag(p.status, VT_DEV_BAD_PAGE);
-        if (pidA < 0 || pidA >= p.num_pages) pidA = -1;
-        if (pidB < 0 || pidB >= p.num_pages) pidB = -1;
-      }
-      if (lane < myrows) s_pids[warp + NW * lane] = pidA;
-      if (lane + 32 < myrows) s_pids[warp + NW * (lane + 32)] = pidB;
-      const float* cbase = p.centroids + (int64_t)h * D;
-      const int64_t cstride = (int64_t)p.Hkv * D;
+      // the rows' page ids for the top-k's emit (the previous item's top-k has passed its
+      // closing barrier)
+      if (lane < it.myrows) s_pids[warp + NW * lane] = pidA;
+      if (lane + 32 < it.myrows) s_pids[warp + NW * (lane + 32)] = pidB;
       const uint32_t ring = region_u32 + warp * kScanRing * 8 * S::C_ROW;
-      const int batches = (myrows + 7) / 8;
-      constexpr int CPRS = S::C_ROW / 16;  // 16-byte chunks per centroid row
-      auto issue = [&](int bt) {
-        if (bt < batches) {
-          const uint32_t dst = ring + (bt % kScanRing) * 8 * S::C_ROW;
-#pragma unroll
-          for (int t8 = 0; t8 < 8; ++t8) {
-            const int i = bt * 8 + t8;  // uniform, < 64
-            const int pg = __shfl_sync(kFull, i < 32 ? pidA : pidB, i & 31);
-#pragma unroll
-            for (int kk = lane; kk < CPRS; kk += 32)
-              if (pg >= 0)
-                cp_async16(dst + t8 * S::C_ROW + kk * 16, cbase + (int64_t)pg * cstride + kk * 4, 16);
-          }
-        }
-        cp_async_commit();
-      };
       uint32_t klo = 0xffffffffu, khi = 0u;  // range of the keys this lane stores
-#pragma unroll
-      for (int bt = 0; bt < kScanRing - 1; ++bt) issue(bt);
-      for (int bt = 0; bt < batches; ++bt) {
-        issue(bt + kScanRing - 1);
+      for (int bt = 0; bt < it.batches; ++bt) {
+        scan_issue(it, bt + kScanRing - 1);
+        // the next item is claimed as warp 0's last batch lands (warp 0 has the most rows),
+        // so that the claim's latency hides under it
+        if (tid == 0 && bt == it.batches - 1) next = claim();
         cp_async_wait<kScanRing - 1>();
         __syncwarp();
         const uint32_t src = ring + (bt % kScanRing) * 8 * S::C_ROW;
@@ -367,7 +405,7 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
         exchange_reduce<SN, LPR_S>(v, lane);
         const int i = bt * 8 + exchange_index<SN, LPR_S>(lane) * RPS + sub;
         const int pg = page_of_lane(pidA, pidB, i);
-        if ((ch % (LPR_S / SN)) == 0 && i < myrows) {
+        if ((ch % (LPR_S / SN)) == 0 && i < it.myrows) {
           const uint32_t key = score_key(pg >= 0 ? v[0] : -INFINITY);
           s_keys[warp + NW * i] = key;
           klo = min(klo, key);
@@ -376,19 +414,29 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
         __syncwarp();  // every lane is done with the slot before it is refilled
       }
       cp_async_wait<0>();
-      if (tid == 0) next = claim();
+      if (tid == 0 && next < 0) next = claim();
       klo = __reduce_min_sync(kFull, klo);
       khi = __reduce_max_sync(kFull, khi);
       if (lane == 0) {
         s_misc[16 + warp] = (int)klo;
         s_misc[16 + NW + warp] = (int)khi;
       }
-      // the top-k scratch lies in warp 0's ring, which only warp 0 has used
-      unsigned char* tk = region;
       if (warp == 0)
         for (int i = lane; i < SmallTopk<NT>::HIST / 4; i += 32)
           reinterpret_cast<int4*>(tk)[i] = make_int4(0, 0, 0, 0);
+      if (tid == 0) s_misc[0] = next;
       __syncthreads();  // all scores of the chunk are in s_keys; the rings are free
+      // A scan item next: its page ids and query mean are fetched and its first batches put
+      // in flight now, so that they land while this chunk's top-k runs.
+      const int t2 = s_misc[0];
+      prepared = t2 < scan_items;
+      if (prepared) {
+        const ScanItem it2 = scan_item(t2);
+        scan_fetch(it2);
+#pragma unroll
+        for (int bt = 0; bt < kScanRing - 1; ++bt) scan_issue(it2, bt);
+      }
+      next = t2;
       klo = 0xffffffffu;
       khi = 0u;
 #pragma unroll
@@ -397,17 +445,17 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
         khi = max(khi, (uint32_t)s_misc[16 + NW + k]);
       }
       // exact top-kc of the chunk, stored in ascending page order
-      const int kc = min(gm.kc, cnt);
-      const int64_t cb = ((int64_t)u * gm.nch_max + c) * gm.kc;
+      const int kc = min(gm.kc, it.cnt);
+      const int64_t cb = ((int64_t)it.u * gm.nch_max + it.c) * gm.kc;
       uint32_t* ck = w.ckey + cb;
       uint16_t* co = w.coff + cb;
       int32_t* cp = w.cpid + cb;
-      small_topk<NT>(s_keys, cnt, kc, klo, khi, tk, [&](int j, int pos) {
+      small_topk<NT>(s_keys, it.cnt, kc, klo, khi, tk, [&](int j, int pos) {
         ck[pos] = s_keys[j];
         co[pos] = (uint16_t)j;
         cp[pos] = s_pids[j];
       });
-      pending = w.unit_done + u;  // counted after the item's closing barrier
+      pending = w.unit_done + it.u;  // counted after the item's closing barrier
     } else {
       // ---------------------------------------------------------------- attention item
       const int a = t - scan_items;
@@ -437,7 +485,7 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
           if (ld_acquire(w.unit_done + u) < nch) {
             const unsigned long long t0 = global_ns();
             for (;;) {
-              __nanosleep(128);
+              __nanosleep(32);
               if (ld_acquire(w.unit_done + u) >= nch) break;
               if (global_ns() - t0 > kWaitNs) {
                 flag(p.status, kDevTimeout);
@@ -454,8 +502,7 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
       if (ok) {
         // ---- the logical pages of this piece into s_sel[0, np), their page ids into s_phys
         const int32_t* ptrow = p.page_table + (int64_t)b * p.pt_stride;
-        auto phys_of = [&](int lp) {
-          int pg = ptrow[lp];
+        auto checked = [&](int pg) {
           if (pg < 0 || pg >= p.num_pages) {
             flag(p.status, VT_DEV_BAD_PAGE);
             pg = -1;
@@ -469,12 +516,15 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
           const int C = (nch - 1) * kc + min(kc, m - (nch - 1) * kChunk);
           const int64_t cb = (int64_t)u * gm.nch_max * kc;  // chunks are contiguous
           const int bos = p.bos, topk = p.topk;
-          for (int q = tid; q < np; q += NT) {  // reserved pages of the piece
-            const int pos = j0 + q;
+          // thread q < np: the piece's q-th page if it is a reserved one (np <= NT).  Its page
+          // id is loaded now and checked only once the candidates' loads below are issued, so
+          // that both take one round trip.
+          int rlp = -1, rpg = -1;
+          if (tid < np) {
+            const int pos = j0 + tid;
             if (pos < bos || pos >= bos + topk) {
-              const int lp = pos < bos ? pos : n - p.eos + (pos - bos - topk);
-              s_sel[q] = lp;
-              s_phys[q] = phys_of(lp);
+              rlp = pos < bos ? pos : n - p.eos + (pos - bos - topk);
+              rpg = ptrow[rlp];
             }
           }
           if (write_sel) {
@@ -491,15 +541,39 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
             unsigned char* tk = region + 6 * NT * 4;
             for (int i = tid; i < SmallTopk<NT>::HIST / 4; i += NT)
               reinterpret_cast<int4*>(tk)[i] = make_int4(0, 0, 0, 0);
+            // candidates tid and tid + NT: every load in flight before any is used
+            const bool h0 = tid < C, h1 = tid + NT < C;
+            uint32_t key0 = 0, key1 = 0;
+            int off0 = 0, off1 = 0, pid0 = -1, pid1 = -1;
+            if (h0) {
+              key0 = __ldcg(w.ckey + cb + tid);
+              off0 = __ldcg(w.coff + cb + tid);
+              pid0 = __ldcg(w.cpid + cb + tid);
+            }
+            if (h1) {
+              key1 = __ldcg(w.ckey + cb + tid + NT);
+              off1 = __ldcg(w.coff + cb + tid + NT);
+              pid1 = __ldcg(w.cpid + cb + tid + NT);
+            }
+            if (rlp >= 0) {
+              s_sel[tid] = rlp;
+              s_phys[tid] = checked(rpg);
+            }
             uint32_t klo = 0xffffffffu, khi = 0u;
-            for (int j = tid; j < C; j += NT) {
-              const uint32_t key = __ldcg(w.ckey + cb + j);
-              const int lp = bos + (j / kc) * kChunk + __ldcg(w.coff + cb + j);
-              keys[j] = key;
-              lps[j] = lp;
-              pids[j] = __ldcg(w.cpid + cb + j);
-              klo = min(klo, key);
-              khi = max(khi, key);
+            if (h0) {
+              keys[tid] = key0;
+              lps[tid] = bos + (tid / kc) * kChunk + off0;
+              pids[tid] = pid0;
+              klo = key0;
+              khi = key0;
+            }
+            if (h1) {
+              const int j = tid + NT;
+              keys[j] = key1;
+              lps[j] = bos + (j / kc) * kChunk + off1;
+              pids[j] = pid1;
+              klo = min(klo, key1);
+              khi = max(khi, key1);
             }
             klo = __reduce_min_sync(kFull, klo);
             khi = __reduce_max_sync(kFull, khi);
@@ -528,6 +602,7 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
             });
             have_phys = true;
           } else {
+            if (rlp >= 0) s_sel[tid] = rlp;  // page ids of the whole piece are looked up below
             uint32_t* keys = reinterpret_cast<uint32_t*>(region);
             uint16_t* offs = reinterpret_cast<uint16_t*>(region + align16(gm.cmax * 4));
             int* hist = reinterpret_cast<int*>(region + align16(gm.cmax * 4) + align16(gm.cmax * 2));
@@ -555,7 +630,7 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
         }
         __syncthreads();
         if (!have_phys) {
-          if (tid < np) s_phys[tid] = phys_of(s_sel[tid]);
+          if (tid < np) s_phys[tid] = checked(ptrow[s_sel[tid]]);
           __syncthreads();
         }
         // ---- warp w: pages w + NW i (i < 4) of the piece through a two-slot ring
@@ -598,44 +673,43 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
         __syncthreads();
         int fin = 1;
         if (A > 1) {
-          if (piece < A - 1) {
-            // publish this piece's partial and move on: the unit's last piece merges them
-            float* dst = w.part + ((int64_t)u * gm.A2 + piece) * G * (D + 2);
-            for (int i = tid; i < G * (D + 2); i += NT) dst[i] = s_cp[i];
-            pending = w.att_cnt + u;
-            fin = 0;
-          } else {
-            // the last piece waits for the other A - 1 partials; their items were claimed
-            // before this one and never wait on a later item, so the wait ends
-            if (tid == 0) {
-              int okm = 1;
-              if (ld_acquire(w.att_cnt + u) < A - 1) {
-                const unsigned long long t0 = global_ns();
-                for (;;) {
-                  __nanosleep(64);
-                  if (ld_acquire(w.att_cnt + u) >= A - 1) break;
-                  if (global_ns() - t0 > kWaitNs) {
-                    flag(p.status, kDevTimeout);
-                    okm = 0;
-                    break;
-                  }
-                }
+          // every piece publishes its partial and counts itself; the piece that arrives last
+          // merges all A of them, so no piece ever waits for another
+          float* dst = w.part + ((int64_t)u * gm.A2 + piece) * G * (D + 2);
+          for (int i = tid; i < G * (D + 2); i += NT) dst[i] = s_cp[i];
+          __syncthreads();
+          if (tid == 0) {
+            // release: the CTA's partial stores (ordered by the barrier); acquire: the partials
+            // of the pieces counted before
+            const int before = atom_acq_rel_add(w.att_cnt + u, 1);
+            s_misc[1] = before == A - 1;
+          }
+          __syncthreads();
+          fin = s_misc[1];
+          if (fin) {
+            // the A partials into s_all (this piece's own from s_cp), eight loads in flight
+            // per thread
+            const float* src = w.part + (int64_t)u * gm.A2 * G * (D + 2);
+            const int tot = A * G * (D + 2), own0 = piece * G * (D + 2), own1 = own0 + G * (D + 2);
+            for (int i0 = 0; i0 < tot; i0 += 8 * NT) {
+              float v[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int i = i0 + k * NT + tid;
+                v[k] = i < tot && (i < own0 || i >= own1) ? __ldcg(src + i) : 0.0f;
               }
-              s_misc[1] = okm;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int i = i0 + k * NT + tid;
+                if (i < tot) s_all[i] = i >= own0 && i < own1 ? s_cp[i - own0] : v[k];
+              }
             }
             __syncthreads();
-            fin = s_misc[1];
-            if (fin) {
-              const float* src = w.part + (int64_t)u * gm.A2 * G * (D + 2);
-              for (int i = tid; i < (A - 1) * G * (D + 2); i += NT) s_all[i] = __ldcg(src + i);
-              for (int i = tid; i < G * (D + 2); i += NT) s_all[(A - 1) * G * (D + 2) + i] = s_cp[i];
-              __syncthreads();
-              merge_partials<G, D>(s_all, A, s_cp, tid, NT);
-              __syncthreads();
-              if (tid == 0) {  // every piece of u is past its waits: reset u's counters
-                w.att_cnt[u] = 0;
-                w.unit_done[u] = 0;
-              }
+            merge_partials<G, D>(s_all, A, s_cp, tid, NT);
+            __syncthreads();
+            if (tid == 0) {  // every piece of u is past its waits: reset u's counters
+              w.att_cnt[u] = 0;
+              w.unit_done[u] = 0;
             }
           }
         } else if (tid == 0 && nch > 0) {
@@ -656,9 +730,8 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
     if (tid == 0) s_misc[0] = next >= 0 ? next : claim();
     __syncthreads();
     if (tid == 0 && pending != nullptr) {
-      // the barrier above ordered every thread's stores of the item before this fence
-      __threadfence();
-      atomicAdd(pending, 1);
+      // the barrier above ordered every thread's stores of the item before this release
+      red_release_add(pending, 1);
       pending = nullptr;
     }
   }
