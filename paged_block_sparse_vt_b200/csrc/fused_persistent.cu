@@ -272,10 +272,6 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
   const int u_split = w.units / 2;  // units from here on take gm.A2 pieces
   const int total_items = scan_items + u_split * gm.A + (w.units - u_split) * gm.A2;
 
-  // A counter that thread 0 bumps (release) once the CTA has passed the barrier at the end
-  // of the item that produced the counted data.
-  int32_t* pending = nullptr;
-
   // ---- scan items: where an item's rows lie, and its per-lane state.  A scan item whose
   // predecessor was a scan item finds its page ids and query mean already in registers and
   // its first kScanRing - 1 batches in flight (prepared during the predecessor's top-k).
@@ -308,19 +304,32 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
   bool prepared = false;
   int pidA = -1, pidB = -1;  // lane l: page ids of its warp's rows l and l + 32
   float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);  // fp32 group mean of q, this lane's float4
-  auto scan_fetch = [&](const ScanItem& it) {
+  // The query rows are loaded ahead with the page ids only for small groups (registers).
+  constexpr bool kQAhead = G <= 2;
+  uint2 qraw[G];  // this lane's 4 query values of each head of the group, as loaded
+  auto load_q = [&](const ScanItem& it) {
     const __nv_bfloat16* q0 = p.q + ((int64_t)it.b * p.Hq + (int64_t)it.h * G) * D + ch * 4;
+#pragma unroll
+    for (int j = 0; j < G; ++j) qraw[j] = *reinterpret_cast<const uint2*>(q0 + (int64_t)j * D);
+  };
+  // loads of an item's page ids (and query rows), not yet used, so that they may be in
+  // flight while other work proceeds ...
+  auto scan_load = [&](const ScanItem& it) {
     const int32_t* ptrow = p.page_table + (int64_t)it.b * p.pt_stride + p.bos + it.c0 + warp;
     pidA = lane < it.myrows ? ptrow[NW * lane] : -1;
     pidB = lane + 32 < it.myrows ? ptrow[NW * (lane + 32)] : -1;
+    if (kQAhead) load_q(it);
+  };
+  // ... and their use: the fp32 group mean, and the page ids checked
+  auto scan_check = [&](const ScanItem& it) {
+    if (!kQAhead) load_q(it);
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < G; ++j) {
-      const uint2 raw = *reinterpret_cast<const uint2*>(q0 + (int64_t)j * D);
-      a.x += bf_lo(raw.x);
-      a.y += bf_hi(raw.x);
-      a.z += bf_lo(raw.y);
-      a.w += bf_hi(raw.y);
+      a.x += bf_lo(qraw[j].x);
+      a.y += bf_hi(qraw[j].x);
+      a.z += bf_lo(qraw[j].y);
+      a.w += bf_hi(qraw[j].y);
     }
     qv = make_float4(a.x / (float)G, a.y / (float)G, a.z / (float)G, a.w / (float)G);
     if (pidA >= p.num_pages || pidA < -1 || pidB >= p.num_pages || pidB < -1 ||
@@ -371,7 +380,8 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
       // ---------------------------------------------------------------- scan item
       const ScanItem it = scan_item(t);
       if (!prepared) {
-        scan_fetch(it);
+        scan_load(it);
+        scan_check(it);
 #pragma unroll
         for (int bt = 0; bt < kScanRing - 1; ++bt) scan_issue(it, bt);
       }
@@ -426,16 +436,12 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
           reinterpret_cast<int4*>(tk)[i] = make_int4(0, 0, 0, 0);
       if (tid == 0) s_misc[0] = next;
       __syncthreads();  // all scores of the chunk are in s_keys; the rings are free
-      // A scan item next: its page ids and query mean are fetched and its first batches put
-      // in flight now, so that they land while this chunk's top-k runs.
+      // A scan item next: the loads of its page ids and query rows are issued now and land
+      // while this chunk's top-k runs; its first batches follow the top-k.
       const int t2 = s_misc[0];
       prepared = t2 < scan_items;
-      if (prepared) {
-        const ScanItem it2 = scan_item(t2);
-        scan_fetch(it2);
-#pragma unroll
-        for (int bt = 0; bt < kScanRing - 1; ++bt) scan_issue(it2, bt);
-      }
+      const ScanItem it2 = scan_item(prepared ? t2 : t);
+      if (prepared) scan_load(it2);
       next = t2;
       klo = 0xffffffffu;
       khi = 0u;
@@ -455,7 +461,16 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
         co[pos] = (uint16_t)j;
         cp[pos] = s_pids[j];
       });
-      pending = w.unit_done + it.u;  // counted after the item's closing barrier
+      // count the chunk as soon as its candidates are stored (the barrier orders every
+      // thread's stores before thread 0's release), then put the next chunk's first batches
+      // in flight
+      __syncthreads();
+      if (tid == 0) red_release_add(w.unit_done + it.u, 1);
+      if (prepared) {
+        scan_check(it2);
+#pragma unroll
+        for (int bt = 0; bt < kScanRing - 1; ++bt) scan_issue(it2, bt);
+      }
     } else {
       // ---------------------------------------------------------------- attention item
       const int a = t - scan_items;
@@ -729,11 +744,6 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
     }
     if (tid == 0) s_misc[0] = next >= 0 ? next : claim();
     __syncthreads();
-    if (tid == 0 && pending != nullptr) {
-      // the barrier above ordered every thread's stores of the item before this release
-      red_release_add(pending, 1);
-      pending = nullptr;
-    }
   }
 
 }
