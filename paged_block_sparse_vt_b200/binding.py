@@ -62,6 +62,9 @@ _lib = None
 def load_library(path: str = LIB_PATH):
     """Load libvt.so (once).  Raises VtError if it is missing: there is no fallback."""
     global _lib
+    lib = _lib
+    if lib is not None:
+        return lib
     with _lock:
         if _lib is None:
             if not os.path.exists(path):
@@ -109,7 +112,13 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else t.data_ptr()
 
 
+# The current stream's handle without building a torch.cuda.Stream object per call.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(t: torch.Tensor) -> int:
+    if _raw_stream is not None:
+        return _raw_stream(t.get_device())
     return torch.cuda.current_stream(t.device).cuda_stream
 
 

@@ -75,4 +75,24 @@ inline cudaError_t ensure_smem_optin(Kernel kern, int bytes, bool nonportable_cl
   return cudaSuccess;
 }
 
+// CTAs of kern per SM at this block size and dynamic shared memory, cached per device for
+// the last size asked for (the occupancy query otherwise costs host time on every call).
+template <typename Kernel>
+inline cudaError_t blocks_per_sm(Kernel kern, int threads, int bytes, std::atomic<long long>* cache,
+                                 int* per_sm) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::atomic<long long>& slot = cache[dev & 63];
+  const long long have = slot.load(std::memory_order_acquire);
+  if (have != 0 && (int)(have >> 32) == bytes) {
+    *per_sm = (int)(have & 0xffffffffLL);
+    return cudaSuccess;
+  }
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kern, threads, bytes);
+  if (e != cudaSuccess) return e;
+  slot.store(((long long)bytes << 32) | (long long)(unsigned)*per_sm, std::memory_order_release);
+  return cudaSuccess;
+}
+
 }  // namespace vt

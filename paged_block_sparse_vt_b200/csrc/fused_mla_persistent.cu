@@ -846,8 +846,9 @@ static cudaError_t launch_mla_persist_t(const DecodeParams& p, const MpWs& w, in
   static std::atomic<int> optin[64];
   cudaError_t e = ensure_smem_optin(kern, smem, false, optin);
   if (e != cudaSuccess) return e;
+  static std::atomic<long long> occ[64];
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kMpThreads, smem);
+  e = blocks_per_sm(kern, kMpThreads, smem, occ, &per_sm);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   cudaLaunchConfig_t cfg = {};
