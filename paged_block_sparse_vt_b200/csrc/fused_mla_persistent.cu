@@ -33,7 +33,7 @@ constexpr int kMpWarps = kMpThreads / 32;
 constexpr int kMpD = 576;
 constexpr int kMpDv = 512;
 constexpr int kMpRow = kMpD + 8;   // smem row stride of Q and K tiles (elements): conflict-free ldmatrix
-constexpr int kMlaChunk = 128;     // candidate pages per scan item (16 per warp)
+constexpr int kMlaChunk = 224;     // candidate pages per scan item (28 per warp)
 constexpr int kMpScanRows = 2;     // centroid rows per ring slot
 constexpr int kMpScanSlots = 5;    // ring slots per warp (4 landing while one is used)
 constexpr int kMpPiece = 8;        // most selected pages per attention item (one warp each)
@@ -182,6 +182,7 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
   constexpr int T = kMpPiece * kPage;
   constexpr int PST = T + 8;
   static_assert(G == 16 || G == 32, "MLA path covers 16 or 32 query heads");
+  static_assert(kMlaChunk <= 32 * kMpWarps, "one page id per lane: at most 32 rows per warp");
   static_assert(kMpPiece >= 2, "the page-max table [kMpPiece][G] holds the merge's [G][2]");
   static_assert(SmallTopk<NT>::BYTES <= kMpScanSlots * kMpScanRows * RB,
                 "the chunk top-k scratch fits in warp 0's ring");
@@ -292,7 +293,7 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
       const int m = n - p.bos - p.eos;
       const int c0 = c * kMlaChunk, cnt = min(kMlaChunk, m - c0);
       const int32_t* ptrow = p.page_table + (int64_t)b * p.pt_stride;
-      // warp w: rows w + NW i (i < 16) of the chunk; lane i < 16 holds the page id of row i
+      // warp w: rows w + NW i (i < 28) of the chunk; lane i < 28 holds the page id of row i
       const int myrows = (cnt - warp + NW - 1) / NW;
       int pid = -1;
       if (lane < myrows) {
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
           const uint32_t dst = ring + (bt % kMpScanSlots) * kMpScanRows * RB;
 #pragma unroll
           for (int rr = 0; rr < kMpScanRows; ++rr) {
-            const int i = bt * kMpScanRows + rr;  // uniform, < 16
+            const int i = bt * kMpScanRows + rr;  // uniform, < 28
             const int pg = __shfl_sync(kFull, pid, i & 31);
             if (i < myrows && pg >= 0) {
               const float* crow = p.centroids + (int64_t)pg * D;
