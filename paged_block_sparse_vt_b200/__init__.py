@@ -8,6 +8,7 @@ library raises ``VtError`` -- there is no CPU or PyTorch fallback.
 from .binding import (  # noqa: F401
     EXPORTS,
     PAGE_SIZE,
+    PreparedCall,
     VT_DEV_BAD_LEN,
     VT_DEV_BAD_ORDER,
     VT_DEV_BAD_PAGE,
@@ -16,6 +17,8 @@ from .binding import (  # noqa: F401
     VtError,
     fused_workspace,
     load_library,
+    prepare_build_centroids,
+    prepare_sparse_decode_fused,
     vt_abi_version,
     vt_build_centroids,
     vt_fused_workspace_size,

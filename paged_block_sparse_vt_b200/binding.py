@@ -296,5 +296,79 @@ def vt_plan_requests(seq_lens: torch.Tensor, order: Optional[torch.Tensor] = Non
     return order
 
 
+class PreparedCall:
+    """One C entry point bound to fixed tensors: the arguments are checked and marshalled
+    once, and each ``run()`` only launches (on the current stream).
+
+    For a serving loop that calls the same operation on the same buffers every step (inputs
+    refreshed in place, as with CUDA graphs).  The bound tensors must keep their storage,
+    shapes and strides for the object's lifetime; it holds references to them.
+    """
+
+    def __init__(self, fn, args, device_index: int, where: str, keep, result):
+        self._fn = fn
+        self._args = args
+        self._dev = device_index
+        self._where = where
+        self._keep = keep
+        self.result = result
+
+    def run(self):
+        stream = _raw_stream(self._dev) if _raw_stream is not None else \
+            torch.cuda.current_stream(self._dev).cuda_stream
+        rc = self._fn(*self._args, stream)
+        if rc != VT_OK:
+            _check(rc, self._where)
+        return self.result
+
+
+def prepare_build_centroids(k_pool: torch.Tensor, pages: torch.Tensor, centroids: torch.Tensor,
+                            status: Optional[torch.Tensor] = None) -> PreparedCall:
+    """vt_build_centroids bound to these tensors; ``run()`` returns ``centroids``."""
+    lib = load_library()
+    _need(pages, "pages", torch.int32, contiguous=True)
+    _need(centroids, "centroids", torch.float32, contiguous=True)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    kv = paged_kv(k_pool, k_pool)
+    P = ctypes.c_void_p
+    args = (ctypes.byref(kv), P(pages.data_ptr()), ctypes.c_int32(pages.numel()),
+            P(centroids.data_ptr()), P(_ptr(status)))
+    return PreparedCall(lib.vt_build_centroids, args, k_pool.get_device(), "vt_build_centroids",
+                        (kv, k_pool, pages, centroids, status), centroids)
+
+
+def prepare_sparse_decode_fused(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos,
+                                eos, sm_scale, out, lse=None, sel=None, n_sel=None, order=None,
+                                status=None, head_dim_v=None, workspace=None) -> PreparedCall:
+    """vt_sparse_decode_fused bound to these tensors; ``run()`` returns (out, lse, sel, n_sel).
+
+    ``out`` (and ``lse`` if wanted) must be given; ``workspace`` as for the unprepared call
+    (from fused_workspace(); required when the shapes need one).
+    """
+    lib = load_library()
+    kv = paged_kv(k_pool, v_pool, head_dim_v)
+    a = decode_args(q, page_table, seq_lens, centroids, topk, bos, eos, sm_scale, order, status)
+    _need(out, "out", torch.bfloat16, contiguous=True)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, contiguous=True)
+    for t, name in ((sel, "sel"), (n_sel, "n_sel")):
+        if t is not None:
+            _need(t, name, torch.int32, contiguous=True)
+    need = int(lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(a)))
+    if need:
+        if workspace is None:
+            raise VtError(VT_ERR_INVALID_ARG, "workspace", f"{need} bytes needed (fused_workspace())")
+        _need(workspace, "workspace", torch.uint8, contiguous=True)
+    P = ctypes.c_void_p
+    args = (ctypes.byref(kv), ctypes.byref(a), P(out.data_ptr()), P(_ptr(lse)), P(_ptr(sel)),
+            P(_ptr(n_sel)), P(_ptr(workspace)),
+            ctypes.c_size_t(0 if workspace is None else workspace.numel()))
+    keep = (kv, a, q, k_pool, v_pool, page_table, seq_lens, centroids, out, lse, sel, n_sel,
+            order, status, workspace)
+    return PreparedCall(lib.vt_sparse_decode_fused, args, q.get_device(), "vt_sparse_decode_fused",
+                        keep, (out, lse, sel, n_sel))
+
+
 def vt_abi_version() -> int:
     return int(load_library().vt_abi_version())
