@@ -246,13 +246,14 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
   // Queue order: block b holds the scan chunks of request b followed by the attention pieces
   // of request b - lag, and the pieces of the last lag requests come at the end.  The
   // attention (tensor-core bound here) then overlaps the scans (HBM bound) of later requests,
-  // and a request's chunks are about three rounds of CTAs ahead of its pieces (measured on the
-  // 64-request latent workload: 1 round 108 us, 2 rounds 104 us, 3 rounds 103 us).  Every
-  // wait is still for items earlier in the queue.
+  // and a request's chunks are about five rounds of CTAs ahead of its pieces (measured on the
+  // 64-request latent workload with 224-page chunks: 1 round 107.2 us, 2 rounds 95.6, 3 rounds
+  // 93.9, 5 rounds 93.1, 8 rounds 93.2, every scan first 93.4).  Every wait is still for items
+  // earlier in the queue.
   const int scan_items = s_prefix[p.B];
   const int A = gm.A;
   const int avg = (scan_items + p.B - 1) / p.B;
-  const int lag = min(p.B, 3 * ((int)gridDim.x / (avg + A) + 1));  // ~3 rounds of CTAs
+  const int lag = min(p.B, 5 * ((int)gridDim.x / (avg + A) + 1));  // ~5 rounds of CTAs
   const int total_items = scan_items + p.B * A;
   auto block_start = [&](int b) { return s_prefix[b] + A * max(0, b - lag); };
 
