@@ -368,11 +368,35 @@ def run_ours(args, world, rank, local):
                                   order=d["order"] if args.plan else None, status=d["status"],
                                   workspace=d["ws"], head_dim_v=c.Dv)
 
-    def step(d):
-        vt.vt_build_centroids(d["k_pool"], d["fill_pages"], d["cent"], status=d["status"])
+    # A page that fills at this step is its request's reserved last page (eos >= 1) until the
+    # next step, so no score of this step reads its centroid: its build runs on a second
+    # stream beside this step's fused call, and the stream joins again before the next step.
+    side = torch.cuda.Stream(dev) if c.eos >= 1 else None
+
+    def build_call(d, prepared=False):
+        if prepared:
+            d["p_build"].run()
+        else:
+            vt.vt_build_centroids(d["k_pool"], d["fill_pages"], d["cent"], status=d["status"])
+
+    def step(d, prepared=False, after_fused=None, overlap=True):
+        main = torch.cuda.current_stream(dev)
+        if side is not None and overlap:
+            side.wait_stream(main)  # this step's inputs are in place
+            with torch.cuda.stream(side):
+                build_call(d, prepared)
+        else:
+            build_call(d, prepared)
         if args.plan:
             vt.vt_plan_requests(d["seq_lens"], d["order"])
-        fused(d)
+        if prepared:
+            d["p_fused"].run()
+        else:
+            fused(d)
+        if after_fused is not None:
+            after_fused(d)
+        if side is not None and overlap:
+            main.wait_stream(side)  # the build is done before anything later on this stream
 
     launches_per_step = 2 + (1 if args.plan else 0)
     for i in range(args.warmup):
@@ -435,13 +459,11 @@ def run_ours(args, world, rank, local):
             order=d["order"] if args.plan else None, status=d["status"], head_dim_v=c.Dv,
             workspace=d["ws"])
 
-    def e2e_step(d):  # copies included
+    def e2e_step(d):  # copies included; one stream (eager cross-stream events cost more host
+        # time than the overlap saves)
         d["in_buf"].copy_(in_h, non_blocking=True)
-        d["p_build"].run()
-        if args.plan:
-            vt.vt_plan_requests(d["seq_lens"], d["order"])
-        d["p_fused"].run()
-        out_h.copy_(d["out_buf"], non_blocking=True)
+        step(d, prepared=True, overlap=False,
+             after_fused=lambda d: out_h.copy_(d["out_buf"], non_blocking=True))
         stream.synchronize()
 
     for i in range(args.warmup):
@@ -483,6 +505,9 @@ def run_ours(args, world, rank, local):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "timing": "the K steps as one CUDA graph replayed once, CUDA events on the launching stream",
+        "step": ("vt_build_centroids (pages filled this step) on a second stream beside "
+                 "vt_sparse_decode_fused, joined before the next step (e2e: one stream)"
+                 if side is not None else "vt_build_centroids then vt_sparse_decode_fused"),
         "clocks": clk,
         "step_bytes": nbytes,
     }

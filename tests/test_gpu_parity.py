@@ -278,3 +278,36 @@ def test_bad_inputs_set_status_and_spare_other_units(oracle):
                         ref["n_sel"].cuda(), c.sm_scale, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == vt.VT_DEV_BAD_SEL
+
+
+@pytest.mark.parametrize("name", ["c2s", "c4s", "c5s"])
+def test_last_page_centroid_is_never_read(name):
+    """With eos >= 1 a request's last page is reserved, so no score reads its centroid: the
+    fused call gives the same bits with those centroid rows set to NaN.  (This is what lets a
+    serving loop build the centroid of a page that fills at this step beside this step's
+    call, as bench.py does.)"""
+    kw = dict(CASES[name])
+    c = config(kw.pop("cfg"), **kw)
+    assert c.eos >= 1
+    w = make_workload(c)
+    d = to_device(w)
+    cent = torch.zeros((w["P"], c.Hkv, c.D), device="cuda")
+    vt.vt_build_centroids(d["k_pool"], all_full_pages(d), cent)
+    n = (d["seq_lens"].long() + 15) // 16
+    last = d["page_table"][torch.arange(c.B, device="cuda"), n - 1].long()
+    poisoned = cent.clone()
+    poisoned[last] = float("nan")
+    args = (d["q"], d["k_pool"], d["v_pool"], d["page_table"], d["seq_lens"])
+    res = []
+    for cc in (cent, poisoned):
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sel = torch.empty((c.B, c.Hkv, c.kmax), dtype=torch.int32, device="cuda")
+        n_sel = torch.empty((c.B, c.Hkv), dtype=torch.int32, device="cuda")
+        out, lse, _, _ = vt.vt_sparse_decode_fused(*args, cc, c.topk, c.bos, c.eos, c.sm_scale,
+                                                   sel=sel, n_sel=n_sel, status=st,
+                                                   head_dim_v=c.Dv)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        res.append((out.view(torch.int16), lse, sel, n_sel))
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
