@@ -417,6 +417,25 @@ def test_unused_slots_are_never_read(oracle):
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
 
 
+def test_last_page_centroid_is_not_a_candidate(oracle):
+    """With eos >= 1 each request's last page is reserved, never scored (reading S4): the
+    oracle's selection and output do not change when every last page's centroid is NaN."""
+    from paged_block_sparse_vt_b200.workloads import make_workload, config
+    c = config(5, B=12, len_lo=200, len_hi=3000, filled=4)
+    assert c.eos >= 1
+    w = make_workload(c)
+    cent = torch.zeros((w["P"], c.Hkv, c.D))
+    oracle.build_centroids(w["k_pool"], torch.cat([w["prebuilt_pages"], w["fill_pages"]]), cent)
+    n = (w["seq_lens"].long() + PS - 1) // PS
+    last = w["page_table"][torch.arange(c.B), n - 1].long()
+    poisoned = cent.clone()
+    poisoned[last] = float("nan")
+    res = [oracle.decode_step(w["q"], w["k_pool"], w["v_pool"], w["page_table"], w["seq_lens"],
+                              cc, c.topk, c.bos, c.eos, c.sm_scale) for cc in (cent, poisoned)]
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
+
+
 def test_mla_value_is_prefix_of_key_row(oracle):
     """MLA: V = K[:, :512] read from the same pool; equals dense attention with that V."""
     from paged_block_sparse_vt_b200.workloads import make_workload, config
