@@ -204,6 +204,12 @@ size_t vt_fused_workspace_size(const vt_paged_kv* kv, const vt_decode_args* a);
  * launched; shapes that need no workspace (B > 2048) run as
  * vt_sparse_decode_fused does.
  *
+ * The array's device address is looked up (cudaGetSymbolAddress) on every
+ * call, in the current device's current context, so it stays right when a
+ * context is destroyed and created again.  The first call on a device may
+ * load the library's module there: make that first call before any stream
+ * capture on the device.
+ *
  * Races: every call on one device shares the one scratch.  Two calls that can
  * be on the GPU at the same time (different streams with no event ordering
  * them, e.g. from two host threads) take work items from each other's queue:

@@ -9,6 +9,10 @@ The arithmetic lives in ``vt_oracle.c`` (plain C, fp64, OpenMP over
 with ctypes.  Arguments are host torch tensors; bf16 tensors are handed to C as
 their 16-bit patterns.  Every function cites the passage it follows in the C
 source's header.
+
+``kind="f32"`` selects a second build of the same C source with fp32 arithmetic
+(``-DVTO_REAL=float -O3 -march=native``).  It is a timing-only copy for the
+benchmark's CPU baseline, never a correctness reference.
 """
 from __future__ import annotations
 
@@ -23,8 +27,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "vt_oracle.c")
 _LIB = os.path.join(_HERE, "libvt_oracle.so")
+_LIB_F32 = os.path.join(_HERE, "libvt_oracle_f32.so")
 _lock = threading.Lock()
-_lib = None
+_libs = {}
 
 OK, ERR_ARG, ERR_LEN, ERR_PAGE = 0, 1, 2, 3
 
@@ -33,23 +38,28 @@ class OracleError(RuntimeError):
     pass
 
 
-def build(force: bool = False) -> str:
-    """Compile vt_oracle.c into libvt_oracle.so next to it (gcc, -O2, OpenMP)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
-        cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
-               _SRC, "-o", tmp, "-lm"]
+def build(force: bool = False, kind: str = "f64") -> str:
+    """Compile vt_oracle.c next to it: libvt_oracle.so (the fp64 oracle: gcc -O2, no FMA
+    contraction, OpenMP), or with kind="f32" the timing-only fp32 copy libvt_oracle_f32.so."""
+    lib = _LIB if kind == "f64" else _LIB_F32
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(_SRC):
+        tmp = lib + f".tmp{os.getpid()}"
+        if kind == "f64":
+            flags = ["-O2", "-ffp-contract=off"]
+        elif kind == "f32":
+            flags = ["-O3", "-march=native", "-DVTO_REAL=float"]
+        else:
+            raise ValueError(kind)
+        cmd = ["gcc", "-std=c11", *flags, "-fopenmp", "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"]
         subprocess.run(cmd, check=True)
-        os.replace(tmp, _LIB)
-    return _LIB
+        os.replace(tmp, lib)
+    return lib
 
 
-def _load():
-    global _lib
+def _load(kind: str = "f64"):
     with _lock:
-        if _lib is None:
-            build()
-            lib = ctypes.CDLL(_LIB)
+        if kind not in _libs:
+            lib = ctypes.CDLL(build(kind=kind))
             i32, i64, f64, p = ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
             lib.vto_set_threads.argtypes = [ctypes.c_int]
             lib.vto_get_threads.restype = ctypes.c_int
@@ -66,16 +76,17 @@ def _load():
                                             i64, i64, i64, i32, p, i64, p, p, i32, i32, i32, f64,
                                             p, p, p, p]
             lib.vto_decode_step.restype = ctypes.c_int
-            _lib = lib
-    return _lib
+            _libs[kind] = lib
+    return _libs[kind]
 
 
-def set_threads(n: int) -> None:
-    _load().vto_set_threads(int(n))
+def set_threads(n: int, kind: str = "f64") -> None:
+    """Threads of the OpenMP loops (0: the OpenMP default, every core of the affinity mask)."""
+    _load(kind).vto_set_threads(int(n))
 
 
-def get_threads() -> int:
-    return int(_load().vto_get_threads())
+def get_threads(kind: str = "f64") -> int:
+    return int(_load(kind).vto_get_threads())
 
 
 def _ptr(t) -> int:
@@ -103,14 +114,15 @@ def _pool_strides(pool: torch.Tensor):
     return pool.stride(0), pool.stride(1), pool.stride(2)
 
 
-def build_centroids(k_pool: torch.Tensor, pages: torch.Tensor, centroids: torch.Tensor) -> None:
+def build_centroids(k_pool: torch.Tensor, pages: torch.Tensor, centroids: torch.Tensor,
+                    kind: str = "f64") -> None:
     """centroids[p] = mean over the page's tokens of K[p] (fp64 sum, fp32 store), in place."""
     P, page_size, hkv, d = k_pool.shape
     assert centroids.dtype == torch.float32 and centroids.is_contiguous()
     assert tuple(centroids.shape) == (P, hkv, d)
     sk = _pool_strides(k_pool)
     pages = _i32(pages)
-    rc = _load().vto_build_centroids(_ptr(_bits(k_pool)), P, page_size, hkv, d, *sk,
+    rc = _load(kind).vto_build_centroids(_ptr(_bits(k_pool)), P, page_size, hkv, d, *sk,
                                      _ptr(pages), pages.numel(), _ptr(centroids))
     _check(rc, "build_centroids")
 
@@ -154,7 +166,7 @@ def sparse_attention(q, k_pool, v_pool, page_table, seq_lens, sel, n_sel, sm_sca
 
 
 def decode_step(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos, eos, sm_scale,
-                head_dim_v=None):
+                head_dim_v=None, kind: str = "f64"):
     """select_pages followed by sparse_attention.  Returns (sel, n_sel, out, lse)."""
     B, hq, d = q.shape
     P, page_size, hkv, _ = k_pool.shape
@@ -166,7 +178,7 @@ def decode_step(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos, e
     n_sel = torch.empty((B, hkv), dtype=torch.int32)
     out = torch.empty((B, hq, dv), dtype=torch.float64)
     lse = torch.empty((B, hq), dtype=torch.float64)
-    rc = _load().vto_decode_step(_ptr(_bits(q)), B, hq, hkv, d, dv, _ptr(_bits(k_pool)), *sk,
+    rc = _load(kind).vto_decode_step(_ptr(_bits(q)), B, hq, hkv, d, dv, _ptr(_bits(k_pool)), *sk,
                                  _ptr(_bits(v_pool)), *sv, P, page_size, _ptr(page_table),
                                  page_table.shape[1], _ptr(seq_lens), _ptr(centroids), topk, bos,
                                  eos, float(sm_scale), _ptr(sel), _ptr(n_sel), _ptr(out), _ptr(lse))

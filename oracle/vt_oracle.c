@@ -41,8 +41,8 @@
  * fp64 from the stored bf16/fp32 inputs.  Inputs in bf16 are passed as their
  * raw 16-bit patterns (a bf16 value is the upper half of an IEEE binary32).
  */
-#include <math.h>
 #include <stdint.h>
+#include <tgmath.h> /* exp and log follow the argument type (fp64 unless VTO_REAL says otherwise) */
 #include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
@@ -53,6 +53,13 @@
 #define VTO_ERR_ARG 1       /* a size, count or pointer argument is invalid */
 #define VTO_ERR_LEN 2       /* a seq_len is < 1 or needs more pages than the page table holds */
 #define VTO_ERR_PAGE 3      /* a page id is outside [0, num_pages) */
+
+/* The arithmetic type.  fp64 is the oracle; -DVTO_REAL=float builds a timing-only copy that
+ * the benchmark uses as a CPU baseline without the fp64 handicap (never as a reference). */
+#ifndef VTO_REAL
+#define VTO_REAL double
+#endif
+typedef VTO_REAL vto_real;
 
 static int g_threads = 0; /* 0: OpenMP default */
 
@@ -66,12 +73,12 @@ int vto_get_threads(void) {
 #endif
 }
 
-/* bf16 -> fp64.  A bf16 value is the upper 16 bits of a binary32 value. */
-static double bf16_to_f64(uint16_t bits) {
+/* bf16 -> the arithmetic type (exact).  A bf16 value is the upper 16 bits of a binary32. */
+static vto_real bf16_to_f64(uint16_t bits) {
   uint32_t u = ((uint32_t)bits) << 16;
   float f;
   memcpy(&f, &u, sizeof f);
-  return (double)f;
+  return (vto_real)f;
 }
 
 static int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -101,10 +108,10 @@ int vto_build_centroids(const uint16_t* k_pool, int64_t num_pages, int32_t page_
     const int64_t h = r % num_kv_heads;
     float* out = centroids + (p * num_kv_heads + h) * head_dim;
     for (int32_t d = 0; d < head_dim; ++d) {
-      double sum = 0.0;
+      vto_real sum = 0.0;
       for (int32_t t = 0; t < page_size; ++t)
         sum += bf16_to_f64(k_pool[p * sk_p + t * sk_t + h * sk_h + d]);
-      out[d] = (float)(sum / (double)page_size);
+      out[d] = (float)(sum / (vto_real)page_size);
     }
   }
   return VTO_OK;
@@ -115,7 +122,7 @@ int vto_build_centroids(const uint16_t* k_pool, int64_t num_pages, int32_t page_
 /* ------------------------------------------------------------------------ */
 
 typedef struct {
-  double score;
+  vto_real score;
   int32_t index; /* logical page index */
 } vto_cand;
 
@@ -176,7 +183,7 @@ int vto_select_pages(const uint16_t* q, int32_t batch, int32_t num_q_heads,
 
 #pragma omp parallel num_threads(vto_get_threads())
   {
-    double* qm = (double*)malloc(sizeof(double) * (size_t)head_dim);
+    vto_real* qm = (vto_real*)malloc(sizeof(vto_real) * (size_t)head_dim);
     vto_cand* cand = (vto_cand*)malloc(sizeof(vto_cand) * (size_t)pt_stride);
     char* keep = (char*)malloc((size_t)pt_stride);
 #pragma omp for schedule(dynamic, 1)
@@ -194,18 +201,18 @@ int vto_select_pages(const uint16_t* q, int32_t batch, int32_t num_q_heads,
       }
       /* q.mean over the G query heads of this KV head */
       for (int32_t d = 0; d < head_dim; ++d) {
-        double s = 0.0;
+        vto_real s = 0.0;
         for (int32_t j = 0; j < G; ++j)
           s += bf16_to_f64(q[((int64_t)b * num_q_heads + (int64_t)h * G + j) * head_dim + d]);
-        qm[d] = s / (double)G;
+        qm[d] = s / (vto_real)G;
       }
       /* GeMV against the centroid of every middle page */
       int32_t m = 0;
       for (int32_t i = bos; i < n - eos; ++i) {
         const int64_t p = page_table[(int64_t)b * pt_stride + i];
         const float* c = centroids + (p * num_kv_heads + h) * head_dim;
-        double s = 0.0;
-        for (int32_t d = 0; d < head_dim; ++d) s += qm[d] * (double)c[d];
+        vto_real s = 0.0;
+        for (int32_t d = 0; d < head_dim; ++d) s += qm[d] * (vto_real)c[d];
         cand[m].score = s;
         cand[m].index = i;
         ++m;
@@ -276,7 +283,8 @@ int vto_sparse_attention(const uint16_t* q, int32_t batch, int32_t num_q_heads,
 #pragma omp parallel num_threads(vto_get_threads())
   {
     const int64_t max_tokens = (int64_t)kmax * page_size;
-    double* z = (double*)malloc(sizeof(double) * (size_t)(max_tokens > 0 ? max_tokens : 1));
+    vto_real* z = (vto_real*)malloc(sizeof(vto_real) * (size_t)(max_tokens > 0 ? max_tokens : 1));
+    vto_real* acc = (vto_real*)malloc(sizeof(vto_real) * (size_t)(head_dim_v > 0 ? head_dim_v : 1));
     const uint16_t** vrow =
         (const uint16_t**)malloc(sizeof(uint16_t*) * (size_t)(max_tokens > 0 ? max_tokens : 1));
 #pragma omp for schedule(dynamic, 1)
@@ -289,34 +297,35 @@ int vto_sparse_attention(const uint16_t* q, int32_t batch, int32_t num_q_heads,
         const int64_t hq = (int64_t)h * G + j;
         const uint16_t* qrow = q + ((int64_t)b * num_q_heads + hq) * head_dim;
         int64_t T = 0;
-        double zmax = -INFINITY;
+        vto_real zmax = -INFINITY;
         for (int32_t s = 0; s < n_sel[u]; ++s) {
           const int32_t i = sel[u * kmax + s];
           const int64_t p = page_table[(int64_t)b * pt_stride + i];
           const int32_t valid = (i == n - 1) ? L - page_size * (n - 1) : page_size;
           for (int32_t t = 0; t < valid; ++t) {
             const uint16_t* krow = k_pool + p * sk_p + t * sk_t + h * sk_h;
-            double dot = 0.0;
+            vto_real dot = 0.0;
             for (int32_t d = 0; d < head_dim; ++d) dot += bf16_to_f64(qrow[d]) * bf16_to_f64(krow[d]);
-            z[T] = sm_scale * dot;
+            z[T] = (vto_real)sm_scale * dot;
             vrow[T] = v_pool + p * sv_p + t * sv_t + h * sv_h;
             if (z[T] > zmax) zmax = z[T];
             ++T;
           }
         }
         double* o = out + ((int64_t)b * num_q_heads + hq) * head_dim_v;
-        for (int32_t d = 0; d < head_dim_v; ++d) o[d] = 0.0;
-        double l = 0.0;
+        for (int32_t d = 0; d < head_dim_v; ++d) acc[d] = 0.0;
+        vto_real l = 0.0;
         for (int64_t t = 0; t < T; ++t) {
-          const double w = exp(z[t] - zmax);
+          const vto_real w = exp(z[t] - zmax);
           l += w;
-          for (int32_t d = 0; d < head_dim_v; ++d) o[d] += w * bf16_to_f64(vrow[t][d]);
+          for (int32_t d = 0; d < head_dim_v; ++d) acc[d] += w * bf16_to_f64(vrow[t][d]);
         }
-        for (int32_t d = 0; d < head_dim_v; ++d) o[d] = (T > 0) ? o[d] / l : 0.0;
+        for (int32_t d = 0; d < head_dim_v; ++d) o[d] = (T > 0) ? acc[d] / l : 0.0;
         if (lse) lse[(int64_t)b * num_q_heads + hq] = (T > 0) ? zmax + log(l) : -INFINITY;
       }
     }
     free(z);
+    free(acc);
     free((void*)vrow);
   }
   return VTO_OK;

@@ -3,8 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
-#include <cstdlib>
-#include <mutex>
+#include <atomic>
 
 #include "decode_params.cuh"
 
@@ -62,12 +61,6 @@ struct Shape {
   int D, Dv, G;
 };
 
-// Optional integer override from the environment (tuning sweeps); 0 when unset.
-int env_int(const char* name) {
-  const char* v = std::getenv(name);
-  return v ? std::atoi(v) : 0;
-}
-
 vt_status check_kv(const vt_paged_kv* kv) {
   if (!kv) return fail(VT_ERR_INVALID_ARG, "kv descriptor is NULL");
   if (!kv->k_pool || !kv->v_pool) return fail(VT_ERR_INVALID_ARG, "k_pool/v_pool is NULL");
@@ -112,23 +105,22 @@ vt_status classify(const vt_paged_kv* kv, int Hq, Shape* sh) {
   return fail(VT_ERR_UNSUPPORTED, "head shape (%d, %d) has no kernel", D, Dv);
 }
 
+// SMs of the current device, looked up once per device.
 int sm_count() {
-  static int cached = 0;
-  if (cached == 0) {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
-      cached = n;
-    else
-      cached = 148;
-  }
-  return cached;
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::atomic<int>& slot = cached[dev & 63];
+  int n = slot.load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+    return 148;
+  slot.store(n, std::memory_order_relaxed);
+  return n;
 }
 
 // Cluster size: CTAs that share one (request, KV head) unit.
 int pick_cluster(const Shape& sh, int64_t units, int kmax) {
-  const int forced = env_int("VT_CLUSTER_SIZE");
-  if (forced == 1 || forced == 2 || forced == 4 || forced == 8 || forced == 16) return forced;
   if (sh.path == kPathMla) {
     int C = 8;
     while (C < 16 && (kmax + C - 1) / C > mla_max_pages_per_cta()) C *= 2;
@@ -274,23 +266,15 @@ static __device__ __align__(256) unsigned char g_static_scratch[VT_STATIC_SCRATC
 // sit at the same offsets in every call and never overlap another call's data.
 constexpr int64_t kStaticUnitCap = 65536;
 
-constexpr int kMaxDevices = 64;
-std::mutex g_static_mu;
-void* g_static_addr[kMaxDevices];  // device address of g_static_scratch, looked up once per device
-
+// Device address of g_static_scratch in the current device's current context.  In host code
+// the array's name only stands in for it, so it is looked up, and it is looked up on every
+// call rather than cached: a context that is destroyed and created again (cudaDeviceReset)
+// reloads the module, and the array may then sit at another address.
 cudaError_t static_scratch_address(void** addr) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_static_mu);
-  if (g_static_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (e != cudaSuccess) return e;
-    g_static_addr[dev] = p;
-  }
-  *addr = g_static_addr[dev];
+  *addr = p;
   return cudaSuccess;
 }
 

@@ -29,3 +29,15 @@ def oracle():
     import oracle as _oracle
     _oracle.build()
     return _oracle
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Print how many units of each GPU selection swapped a tied page with the oracle's."""
+    try:
+        from parity import REPORTS
+    except Exception:
+        return
+    if REPORTS:
+        terminalreporter.section("selection swaps against the oracle (tie rule)")
+        for line in REPORTS:
+            terminalreporter.write_line(line)

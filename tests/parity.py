@@ -3,21 +3,36 @@
 Tolerances (from the target the method is built to):
   * centroids: |c_gpu - c_ref| <= 1e-5 |c_ref| + 1e-6 (fp32 storage of an fp64 mean);
   * selected pages: identical sets per (request, KV head), except a swap at the top-k
-    boundary between pages whose oracle scores are within 1e-4 relative of the k-th score
-    (relative to max(|s_i|, |s_k|, sum_d |qm_d c_id|): the fp32 GPU score error scales with
-    the magnitude of the terms, not of the possibly cancelling sum);
-  * attention output: max-abs error <= 1e-2 (bf16 output of an fp32 accumulation);
+    boundary between pages whose oracle scores differ from the k-th selected score by at most
+    1e-4 relative.  Two bounds are counted for every swap:
+      strict  -- |s_i - s_k| <= 1e-4 max(|s_i|, |s_k|), the stated tie rule;
+      relaxed -- |s_i - s_k| <= 1e-4 max(|s_i|, |s_k|, sum_d |qm_d c_id|): the error of an
+                 fp32 dot product grows with the magnitude of its terms, not with the sum,
+                 so where the terms cancel (a score near zero) the strict rule asks for more
+                 than fp32 scoring can give.
+    A swap must pass the relaxed bound; the swaps that pass only the relaxed one are counted
+    and reported, and at most MAX_SWAP_FRACTION of the units (plus one) may swap at all;
+  * attention output: max-abs error <= 1e-2 (bf16 output of an fp32 accumulation) on EVERY
+    unit.  A unit whose selection is a tolerated swap is held against the oracle's attention
+    over that selection: a set the oracle's own scores accept as a top-k (every page that
+    differs ties with the k-th score), so it is one of the method's correct answers;
   * lse: abs error <= 1e-3.
 """
 from __future__ import annotations
+
+from dataclasses import dataclass, field
 
 import torch
 
 CENTROID_RTOL, CENTROID_ATOL = 1e-5, 1e-6
 SCORE_RTOL = 1e-4
+MAX_SWAP_FRACTION = 0.01
 OUT_ATOL = 1e-2
 LSE_ATOL = 1e-3
 PS = 16
+
+# selection reports of this session, printed by conftest at the end of the run
+REPORTS: list = []
 
 
 def to_device(w: dict, device="cuda") -> dict:
@@ -70,16 +85,28 @@ def _sigma(w: dict, cent: torch.Tensor, b: int, h: int, i: int) -> float:
     return float((qm * cent[p, h].double()).abs().sum())
 
 
-def compare_selection(w: dict, ref: dict, cent: torch.Tensor, sel: torch.Tensor,
-                      n_sel: torch.Tensor) -> torch.Tensor:
-    """Assert GPU selection == oracle selection up to tolerated boundary swaps.
+@dataclass
+class SelectionReport:
+    """What a GPU selection did against the oracle's."""
+    label: str
+    units: int
+    swapped: list = field(default_factory=list)  # (b, h) units whose set differs (tolerated)
+    swapped_pages: int = 0                       # pages in those differences
+    strict_fail: int = 0                         # of them, accepted by the relaxed bound only
 
-    Returns a bool [B, Hkv] mask of units whose selected set is identical.
-    """
+    def summary(self) -> str:
+        return (f"{self.label}: {self.units} units, {len(self.swapped)} with a tolerated swap "
+                f"({self.swapped_pages} pages; {self.strict_fail} of them pass only the relaxed "
+                f"bound)")
+
+
+def compare_selection(w: dict, ref: dict, cent: torch.Tensor, sel: torch.Tensor,
+                      n_sel: torch.Tensor, label: str = "") -> SelectionReport:
+    """Assert GPU selection == oracle selection up to tolerated boundary swaps, and count them."""
     c = w["config"]
     sel, n_sel = sel.cpu(), n_sel.cpu()
-    same = torch.ones((c.B, c.Hkv), dtype=torch.bool)
     kmax = ref["topk"] + ref["bos"] + ref["eos"]
+    rep = SelectionReport(label=label or c.name, units=c.B * c.Hkv)
     for b in range(c.B):
         n = (int(w["seq_lens"][b]) + PS - 1) // PS
         for h in range(c.Hkv):
@@ -90,33 +117,62 @@ def compare_selection(w: dict, ref: dict, cent: torch.Tensor, sel: torch.Tensor,
             assert all(x == -1 for x in sel[b, h, int(n_sel[b, h]):kmax].tolist())
             if got == want:
                 continue
-            same[b, h] = False
+            rep.swapped.append((b, h))
             s = ref["scores"][b, h]
             chosen = [s[i].item() for i in want if ref["bos"] <= i < n - ref["eos"]]
             kth = min(chosen)
             for i in set(got) ^ set(want):
                 assert ref["bos"] <= i < n - ref["eos"], f"unit {(b, h)}: reserved page {i} differs"
                 si = s[i].item()
-                tol = SCORE_RTOL * max(abs(si), abs(kth), _sigma(w, cent, b, h, i))
+                strict = SCORE_RTOL * max(abs(si), abs(kth))
+                tol = max(strict, SCORE_RTOL * _sigma(w, cent, b, h, i))
                 assert abs(si - kth) <= tol, (
                     f"unit {(b, h)}: page {i} score {si!r} vs k-th {kth!r} (tol {tol:.3g})")
-    return same
+                rep.swapped_pages += 1
+                rep.strict_fail += int(abs(si - kth) > strict)
+    assert len(rep.swapped) <= MAX_SWAP_FRACTION * rep.units + 1, rep.summary()
+    REPORTS.append(rep.summary())
+    return rep
 
 
-def compare_outputs(out: torch.Tensor, lse, ref: dict, mask=None, G: int = 1) -> float:
-    """Max-abs check of out [B,Hq,Dv] (and lse) against the oracle, over units in mask."""
+def reference_outputs(oracle, w: dict, ref: dict, sel: torch.Tensor, n_sel: torch.Tensor,
+                      rep: SelectionReport):
+    """The oracle's out / lse for every unit of the GPU's selection: the oracle's own where the
+    sets agree, and for the requests holding a tolerated swap the oracle's attention over the
+    swapped set (compare_selection has checked that set against the oracle's scores)."""
+    out, lse = ref["out"].clone(), ref["lse"].clone()
+    reqs = sorted({b for b, _ in rep.swapped})
+    if not reqs:
+        return out, lse
+    c = w["config"]
+    it = torch.tensor(reqs)
+    o2, l2 = oracle.sparse_attention(w["q"][it].contiguous(), w["k_pool"], w["v_pool"],
+                                     w["page_table"][it].contiguous(),
+                                     w["seq_lens"][it].contiguous(),
+                                     sel.cpu()[it].contiguous(), n_sel.cpu()[it].contiguous(),
+                                     c.sm_scale, head_dim_v=c.Dv)
+    out[it] = o2
+    lse[it] = l2
+    return out, lse
+
+
+def compare_outputs(out: torch.Tensor, lse, ref_out: torch.Tensor, ref_lse=None) -> float:
+    """Max-abs check of out [B,Hq,Dv] (and lse) against the oracle's, on every row."""
     o = out.cpu().double()
-    r = ref["out"]
-    if mask is not None:
-        rows = mask.repeat_interleave(G, dim=1)  # [B, Hq]
-        o, r = o[rows], r[rows]
     assert torch.isfinite(o).all()
-    err = (o - r).abs().max().item() if o.numel() else 0.0
+    err = (o - ref_out).abs().max().item() if o.numel() else 0.0
     assert err <= OUT_ATOL, f"max abs error {err:.4g} > {OUT_ATOL}"
     if lse is not None:
-        lg, lr = lse.cpu().double(), ref["lse"]
-        if mask is not None:
-            lg, lr = lg[rows], lr[rows]
-        lerr = (lg - lr).abs().max().item() if lg.numel() else 0.0
+        lg = lse.cpu().double()
+        lerr = (lg - ref_lse).abs().max().item() if lg.numel() else 0.0
         assert lerr <= LSE_ATOL, f"lse max abs error {lerr:.4g}"
     return err
+
+
+def check_step(oracle, w: dict, ref: dict, cent_ref: torch.Tensor, sel, n_sel, out, lse,
+               label: str = "") -> SelectionReport:
+    """Selection within the tie rule, then every unit's output and lse against the oracle."""
+    rep = compare_selection(w, ref, cent_ref, sel, n_sel, label=label)
+    ro, rl = reference_outputs(oracle, w, ref, sel, n_sel, rep)
+    compare_outputs(out, lse, ro, rl if lse is not None else None)
+    return rep

@@ -1,38 +1,20 @@
 """Full-size parity: the benchmark workloads at their real sizes, through the calls bench.py
 times (centroid build of the prebuilt and of the newly filled pages, then the fused call on a
-workspace), against the oracle on a sample of requests that it computes one by one.  Every
-request, sampled or not, is also checked through properties that hold at any size.
+workspace), against the oracle on EVERY request (the fp64 oracle runs these sizes in seconds
+on the host cores): every centroid row, every selection within the tie rule, every output
+row and lse.  Every request is also checked through properties that hold at any size.
 
 Pool pages that belong to no request and token slots past the end of each request hold NaN,
 so a gather from the wrong place cannot pass.
 """
-import dataclasses
-
 import pytest
 import torch
 
 import paged_block_sparse_vt_b200 as vt
 from paged_block_sparse_vt_b200.workloads import config, make_workload
-from parity import (PS, check_centroids, compare_outputs, compare_selection, oracle_step,
-                    to_device)
+from parity import PS, all_full_pages, check_centroids, check_step, oracle_step, to_device
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
-
-SAMPLE = 6  # requests per workload the oracle recomputes
-
-
-def _sample(seq_lens: torch.Tensor) -> list:
-    """The longest and the shortest request plus seeded random others."""
-    B = seq_lens.numel()
-    if B <= SAMPLE:
-        return list(range(B))
-    pick = {int(seq_lens.argmax()), int(seq_lens.argmin())}
-    g = torch.Generator().manual_seed(17)
-    for i in torch.randperm(B, generator=g).tolist():
-        if len(pick) == SAMPLE:
-            break
-        pick.add(i)
-    return sorted(pick)
 
 
 def _check_invariants(c, seq_lens, sel, n_sel, out) -> None:
@@ -78,18 +60,10 @@ def test_full_size_fused_against_oracle(cfg, oracle):
     _check_invariants(c, d["seq_lens"], sel, n_sel, out)
     del d
 
-    idx = _sample(w["seq_lens"])
-    it = torch.tensor(idx)
-    sub = dict(w, config=dataclasses.replace(c, B=len(idx)), q=w["q"][it],
-               page_table=w["page_table"][it], seq_lens=w["seq_lens"][it])
-    # the oracle's centroids of the sampled requests' full pages (prebuilt and newly filled)
-    n = (sub["seq_lens"].long() + PS - 1) // PS
-    full = [sub["page_table"][b, : int(n[b]) - (0 if int(sub["seq_lens"][b]) % PS == 0 else 1)]
-            for b in range(len(idx))]
-    pages = torch.cat(full).to(torch.int32)
     cent_ref = torch.full((w["P"], c.Hkv, c.D), float("nan"))
+    pages = all_full_pages(w)
     oracle.build_centroids(w["k_pool"], pages, cent_ref)
     check_centroids(cent, cent_ref, pages)
-    ref = oracle_step(oracle, sub, cent_ref)
-    same = compare_selection(sub, ref, cent_ref, sel[it.cuda()], n_sel[it.cuda()])
-    compare_outputs(out[it.cuda()], lse[it.cuda()], ref, mask=same, G=c.G)
+    del cent
+    ref = oracle_step(oracle, w, cent_ref)
+    check_step(oracle, w, ref, cent_ref, sel, n_sel, out, lse, label=f"full-size config {cfg}")

@@ -11,8 +11,8 @@ import torch
 
 import paged_block_sparse_vt_b200 as vt
 from paged_block_sparse_vt_b200.workloads import config, make_workload
-from parity import (all_full_pages, check_centroids, compare_outputs, compare_selection,
-                    oracle_centroids, oracle_step, to_device)
+from parity import (all_full_pages, check_centroids, check_step, compare_outputs,
+                    compare_selection, oracle_centroids, oracle_step, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -98,7 +98,7 @@ def test_select_pages(name, oracle):
                                     status=st, head_dim_v=c.Dv)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    compare_selection(w, ref, cent_ref, sel, n_sel)
+    compare_selection(w, ref, cent_ref, sel, n_sel, label=f"select {name}")
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -114,7 +114,7 @@ def test_sparse_decode(name, oracle):
                                    c.sm_scale, status=st, head_dim_v=c.Dv)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    compare_outputs(out, lse, ref)
+    compare_outputs(out, lse, ref["out"], ref["lse"])
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -135,15 +135,13 @@ def test_fused_pipeline(name, oracle):
                                                head_dim_v=c.Dv)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    same = compare_selection(w, ref, cent_ref, sel, n_sel)
-    compare_outputs(out, lse, ref, mask=same, G=c.G)
+    check_step(oracle, w, ref, cent_ref, sel, n_sel, out, lse, label=f"fused {name}")
     # the two-launch path (select, then decode) meets the same bar
     sel2, n_sel2 = vt.vt_select_pages(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
                                       d["seq_lens"], cent, c.topk, c.bos, c.eos, head_dim_v=c.Dv)
     out2, lse2 = vt.vt_sparse_decode(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
                                      d["seq_lens"], sel2, n_sel2, c.sm_scale, head_dim_v=c.Dv)
-    same2 = compare_selection(w, ref, cent_ref, sel2, n_sel2)
-    compare_outputs(out2, lse2, ref, mask=same2, G=c.G)
+    check_step(oracle, w, ref, cent_ref, sel2, n_sel2, out2, lse2, label=f"select+decode {name}")
 
 
 @pytest.mark.parametrize("name", ["c2s", "c5s", "g3_d128", "g7_d64"])
@@ -216,8 +214,8 @@ def test_edge_lengths_and_knobs(topk, bos, eos, oracle):
                                                c.sm_scale, sel=sel, n_sel=n_sel, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    same = compare_selection(w, ref, cent_ref, sel, n_sel)
-    compare_outputs(out, lse, ref, mask=same, G=c.G)
+    check_step(oracle, w, ref, cent_ref, sel, n_sel, out, lse,
+               label=f"edge k={topk} bos={bos} eos={eos}")
 
 
 def test_strided_pools_match_contiguous(oracle):

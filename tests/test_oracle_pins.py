@@ -453,3 +453,23 @@ def test_mla_value_is_prefix_of_key_row(oracle):
     assert out.shape == (2, 32, 512)
     assert torch.allclose(out, ref, rtol=0, atol=1e-12)
     assert torch.allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def test_fp32_timing_copy_tracks_the_oracle(oracle):
+    """The fp32 build of the same source (the benchmark's CPU-baseline copy, never a
+    reference) computes the same step: same selections here, outputs within fp32 rounding."""
+    from paged_block_sparse_vt_b200.workloads import config, make_workload
+    w = make_workload(config(2, B=4, len_lo=600, len_hi=3000, pool_pages=1000))
+    c = w["config"]
+    full = torch.cat([w["prebuilt_pages"], w["fill_pages"]]).to(torch.int32)
+    res = []
+    for kind in ("f64", "f32"):
+        cent = torch.zeros((w["P"], c.Hkv, c.D))
+        oracle.build_centroids(w["k_pool"], full, cent, kind=kind)
+        res.append((cent,) + oracle.decode_step(w["q"], w["k_pool"], w["v_pool"], w["page_table"],
+                                                w["seq_lens"], cent, c.topk, c.bos, c.eos,
+                                                c.sm_scale, kind=kind))
+    (c64, s64, n64, o64, l64), (c32, s32, n32, o32, l32) = res
+    assert torch.allclose(c32, c64, rtol=1e-6, atol=1e-7)
+    assert torch.equal(n32, n64) and torch.equal(s32, s64)
+    assert (o32 - o64).abs().max().item() < 1e-4 and (l32 - l64).abs().max().item() < 1e-4
