@@ -81,6 +81,36 @@ def algorithmic_bytes(c, seq_lens: torch.Tensor) -> dict:
                 kv_bytes=c.Hkv * int((2 * (c.D + dv) * tokens).sum()))
 
 
+def variant_bytes(c, seq_lens: torch.Tensor) -> dict:
+    """Algorithmic bytes of the split calls, from the same lengths:
+    select  = q + page-table rows + candidate centroids + sel/n_sel written
+    decode  = q + out + lse + sel/n_sel read + one page-table entry per selected page
+              + the selected K/V rows
+    """
+    L = seq_lens.long()
+    n = (L + PAGE_SIZE - 1) // PAGE_SIZE
+    last_valid = L - PAGE_SIZE * (n - 1)
+    sparse = n > c.kmax
+    cand = torch.where(sparse, n - c.bos - c.eos, torch.zeros_like(n))
+    sel_pages = torch.minimum(n, torch.full_like(n, c.kmax))
+    tokens = PAGE_SIZE * (sel_pages - 1) + last_valid
+    dv = 0 if c.mla else c.Dv
+    q = 2 * c.B * c.Hq * c.D
+    selw = 4 * c.B * c.Hkv * (c.kmax + 1)
+    select = q + 4 * int(n.sum()) + c.Hkv * int((4 * c.D * cand).sum()) + selw
+    decode = (q + 2 * c.B * c.Hq * c.Dv + 4 * c.B * c.Hq + selw
+              + c.Hkv * int((4 * sel_pages + 2 * (c.D + dv) * tokens).sum()))
+    return dict(select=select, decode=decode)
+
+
+def build_bytes(c, pages: int) -> int:
+    """vt_build_centroids over `pages` pages: K rows read, fp32 centroid rows written, ids."""
+    return pages * (PAGE_SIZE * c.Hkv * c.D * 2 + c.Hkv * c.D * 4 + 4)
+
+
+NOMINAL_HBM_GBS = 8000.0
+
+
 def read_peak_hbm():
     try:
         with open(PEAKS_FILE) as f:
@@ -227,7 +257,7 @@ def oracle_prepare(w):
     return cent
 
 
-def oracle_step(w, cent, reqs):
+def oracle_step(w, cent, reqs, kind="f64"):
     """One oracle decode step over the requests in ``reqs``: build the centroids of the pages
     that fill at this step, then select + attend."""
     import oracle
@@ -238,10 +268,11 @@ def oracle_step(w, cent, reqs):
     fill = [int(w["page_table"][b, int(n[i]) - 1]) for i, b in enumerate(reqs)
             if int(L[i]) % PAGE_SIZE == 0]
     if fill:
-        oracle.build_centroids(w["k_pool"], torch.tensor(fill, dtype=torch.int32), cent)
+        oracle.build_centroids(w["k_pool"], torch.tensor(fill, dtype=torch.int32), cent,
+                               kind=kind)
     oracle.decode_step(w["q"][idx].contiguous(), w["k_pool"], w["v_pool"],
                        w["page_table"][idx].contiguous(), L.contiguous(), cent, c.topk, c.bos,
-                       c.eos, c.sm_scale)
+                       c.eos, c.sm_scale, head_dim_v=c.Dv, kind=kind)
 
 
 def oracle_sample_size(w, cent, target_s: float) -> list:
@@ -479,13 +510,31 @@ def run_ours(args, world, rank, local):
     status = max(int(d["status"].item()) for d in reps)
     if status:
         raise SystemExit(f"device status {status}: an input was rejected by the kernels")
+    graph.reset()
+    fused_graph.reset()
+    del reps, graph, fused_graph
+    torch.cuda.empty_cache()
+
+    peak, peak_kind = read_peak_hbm()
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        pc_clocks = ClockSampler(local)
+        pc_clocks.start()
+        per_config = {}
+        for cfg in (1, 2, 3, 4, 5):
+            t0 = time.perf_counter()
+            per_config[str(cfg)] = measure_config(vt, cfg, dev, peak)
+            log(f"config {cfg}: {time.perf_counter() - t0:.1f} s, fused "
+                f"{per_config[str(cfg)]['fused']['us']} us")
+        per_config["clocks"] = pc_clocks.stop()
+        per_config["timing"] = ("per row: 10 calls captured as one CUDA graph, one untimed "
+                                "replay, one replay between CUDA events; us = per call")
 
     if rank != 0:
         return
     ms = elapsed / args.steps * 1e3
     units = c.B * c.Hq
     value = aggregate_value(world, units, args.steps, elapsed)
-    peak, peak_kind = read_peak_hbm()
     achieved = nbytes["fused"] / (fused_ms / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -494,7 +543,10 @@ def run_ours(args, world, rank, local):
         "config": workload_config(c, w, args),
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "traffic": recorded_traffic(args.config),
+            "frac": achieved / peak, "frac_nominal_8000": achieved / NOMINAL_HBM_GBS,
+            "frac_note": ("frac is against the measured copy peak (the roofline's denominator); "
+                          "frac_nominal_8000 against the nominal ~8 TB/s HBM3e figure"),
+            "traffic": recorded_traffic(args.config),
             "kernel": ("persist_mla_kernel" if c.mla else "persist_fused_kernel")
                       + " (vt_sparse_decode_fused)",
             "algorithmic_bytes_per_launch": nbytes["fused"], "kernel_ms": fused_ms,
@@ -511,31 +563,174 @@ def run_ours(args, world, rank, local):
         "clocks": clk,
         "step_bytes": nbytes,
     }
+    if per_config is not None:
+        line["per_config"] = per_config
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------------------------------
+# every workload of the hot-path table: fused launch, split calls, centroid builds
+# ------------------------------------------------------------------------------------------
+def graph_time_ms(calls, iters: int, dev) -> float:
+    """Average ms of one call: `iters` calls (rotating over `calls`) captured as one CUDA graph,
+    replayed once untimed, then once between CUDA events on the launching stream."""
+    for i in range(2):
+        calls[i % len(calls)]()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(iters):
+            calls[i % len(calls)]()
+    g.replay()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    g.replay()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / iters
+    del g
+    return ms
+
+
+def measure_config(vt, cfg: int, dev, peak: float, iters: int = 10) -> dict:
+    """One workload of the hot-path table on this GPU: the fused call (and, where the table
+    asks for them, select-only, decode-only, select + decode back to back, the centroid build
+    of the pages filled this step, and a build of every page of the pool).  Inputs whose
+    per-call bytes are below 4x the 126 MB L2 rotate over copies so that no call finds its data
+    in L2; the tiny workload is launch-bound and runs from L2."""
+    c = config(cfg)
+    w = make_workload(c, seed=1000 + cfg)
+    nb = algorithmic_bytes(c, w["seq_lens"])
+    vb = variant_bytes(c, w["seq_lens"])
+    l2 = 126e6
+    reps = 1 if (nb["fused"] >= 4 * l2 or nb["fused"] < 1e6) else min(3, 1 + int(4 * l2 // nb["fused"]))
+    ds = []
+    for _ in range(reps):
+        d = {k: w[k].to(dev) for k in ("q", "k_pool", "page_table", "seq_lens", "prebuilt_pages",
+                                       "fill_pages")}
+        d["v_pool"] = d["k_pool"] if w["v_pool"] is w["k_pool"] else w["v_pool"].to(dev)
+        d["cent"] = torch.zeros((w["P"], c.Hkv, c.D), dtype=torch.float32, device=dev)
+        vt.vt_build_centroids(d["k_pool"], d["prebuilt_pages"], d["cent"])
+        vt.vt_build_centroids(d["k_pool"], d["fill_pages"], d["cent"])
+        d["out"] = torch.empty((c.B, c.Hq, c.Dv), dtype=torch.bfloat16, device=dev)
+        d["lse"] = torch.empty((c.B, c.Hq), dtype=torch.float32, device=dev)
+        d["sel"] = torch.empty((c.B, c.Hkv, c.kmax), dtype=torch.int32, device=dev)
+        d["n_sel"] = torch.empty((c.B, c.Hkv), dtype=torch.int32, device=dev)
+        d["status"] = torch.zeros((1,), dtype=torch.int32, device=dev)
+        d["ws"] = vt.fused_workspace(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                     d["seq_lens"], d["cent"], c.topk, c.bos, c.eos,
+                                     head_dim_v=c.Dv)
+        ds.append(d)
+    torch.cuda.synchronize(dev)
+
+    def fused(d):
+        return lambda: vt.vt_sparse_decode_fused(
+            d["q"], d["k_pool"], d["v_pool"], d["page_table"], d["seq_lens"], d["cent"], c.topk,
+            c.bos, c.eos, c.sm_scale, out=d["out"], lse=d["lse"], status=d["status"],
+            workspace=d["ws"], head_dim_v=c.Dv)
+
+    def select(d):
+        return lambda: vt.vt_select_pages(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                          d["seq_lens"], d["cent"], c.topk, c.bos, c.eos,
+                                          sel=d["sel"], n_sel=d["n_sel"], status=d["status"],
+                                          head_dim_v=c.Dv)
+
+    def decode(d):
+        return lambda: vt.vt_sparse_decode(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                           d["seq_lens"], d["sel"], d["n_sel"], c.sm_scale,
+                                           out=d["out"], lse=d["lse"], status=d["status"],
+                                           head_dim_v=c.Dv)
+
+    def row(ms, nbytes):
+        gbs = nbytes / (ms / 1e3) / 1e9
+        return {"us": round(ms * 1e3, 2), "bytes": nbytes, "GB_s": round(gbs, 1),
+                "frac": round(gbs / peak, 4), "frac_nominal_8000": round(gbs / NOMINAL_HBM_GBS, 4),
+                "req_heads_per_s": c.B * c.Hq / (ms / 1e3)}
+
+    res = {"workload": f"{c.name} (B={c.B}, Hq={c.Hq}, Hkv={c.Hkv}, D={c.D}/{c.Dv}, context "
+                       f"{lengths_text(c)}, top-{c.topk}+{c.bos}+{c.eos}, pool {w['P']} pages)",
+           "input_copies": reps}
+    res["fused"] = row(graph_time_ms([fused(d) for d in ds], iters, dev), nb["fused"])
+    if cfg in (2, 3):
+        res["select_only"] = row(graph_time_ms([select(d) for d in ds], iters, dev), vb["select"])
+        for d in ds:
+            select(d)()
+        res["decode_only"] = row(graph_time_ms([decode(d) for d in ds], iters, dev), vb["decode"])
+        res["select_then_decode"] = row(
+            graph_time_ms([(lambda d=d: (select(d)(), decode(d)())) for d in ds], iters, dev),
+            vb["select"] + vb["decode"])
+    n_fill = int(w["fill_pages"].numel())
+    if n_fill:
+        d = ds[0]
+        res["build_filled_pages"] = dict(pages=n_fill, **row(graph_time_ms(
+            [lambda: vt.vt_build_centroids(d["k_pool"], d["fill_pages"], d["cent"],
+                                           status=d["status"])], iters, dev),
+            build_bytes(c, n_fill)))
+        res["build_filled_pages"].pop("req_heads_per_s")
+    if cfg == 3:
+        d = ds[0]
+        allp = torch.arange(w["P"], dtype=torch.int32, device=dev)
+        res["build_all_pages"] = dict(pages=w["P"], **row(graph_time_ms(
+            [lambda: vt.vt_build_centroids(d["k_pool"], allp, d["cent"], status=d["status"])],
+            5, dev), build_bytes(c, w["P"])))
+        res["build_all_pages"].pop("req_heads_per_s")
+    torch.cuda.synchronize(dev)
+    if any(int(d["status"].item()) for d in ds):
+        raise SystemExit(f"config {cfg}: device status set: an input was rejected by the kernels")
+    del ds
+    torch.cuda.empty_cache()
+    return res
+
+
 def cpu_baseline(w) -> dict:
-    """The oracle, as it stands, on a bounded sample of the same workload (~15 s of CPU)."""
+    """The oracle, as it stands, on a bounded sample of the same workload (~10 s of CPU on all
+    cores of the affinity mask), plus two labelled variants on smaller samples: the same C
+    source built with fp32 arithmetic and -O3 -march=native (a timing-only copy), and the
+    fp64 oracle on one thread."""
     import oracle
     c = w["config"]
     cent = oracle_prepare(w)
-    reqs = oracle_sample_size(w, cent, target_s=5.0)
-    oracle_step(w, cent, reqs)  # warm
-    t0 = time.perf_counter()
-    reps = 0
-    while reps < 3 or time.perf_counter() - t0 < 10.0:
-        oracle_step(w, cent, reqs)
-        reps += 1
-        if time.perf_counter() - t0 > 30.0:
-            break
-    dt = (time.perf_counter() - t0) / reps
-    return {"value": len(reqs) * c.Hq / dt, "unit": UNIT, "cores": oracle.get_threads(),
-            "kind": "oracle",
-            "sample": f"{reps} oracle steps over requests 0..{len(reqs) - 1} of the same batch "
-                      f"({len(reqs) * c.Hq} req-heads each; build of filled pages + select + "
-                      f"attend), fp64"}
+
+    def timed(reqs, kind, min_s, max_s):
+        oracle_step(w, cent, reqs, kind=kind)  # warm
+        t0 = time.perf_counter()
+        reps = 0
+        while reps < 2 or time.perf_counter() - t0 < min_s:
+            oracle_step(w, cent, reqs, kind=kind)
+            reps += 1
+            if time.perf_counter() - t0 > max_s:
+                break
+        return (time.perf_counter() - t0) / reps, reps
+
+    reqs = oracle_sample_size(w, cent, target_s=3.0)
+    dt, reps = timed(reqs, "f64", 10.0, 30.0)
+    res = {"value": len(reqs) * c.Hq / dt, "unit": UNIT, "cores": oracle.get_threads(),
+           "kind": "oracle",
+           "sample": f"{reps} oracle steps over requests 0..{len(reqs) - 1} of the same batch "
+                     f"({len(reqs) * c.Hq} req-heads each; build of filled pages + select + "
+                     f"attend), fp64"}
+    variants = []
+    dt32, reps32 = timed(reqs, "f32", 3.0, 10.0)
+    variants.append({"value": len(reqs) * c.Hq / dt32, "unit": UNIT,
+                     "cores": oracle.get_threads("f32"),
+                     "kind": "oracle source built with fp32 arithmetic, gcc -O3 -march=native "
+                             "(timing-only copy)",
+                     "sample": f"{reps32} steps over requests 0..{len(reqs) - 1}"})
+    oracle.set_threads(1)
+    try:
+        one = reqs[: max(1, len(reqs) // 8)]
+        dt1, reps1 = timed(one, "f64", 3.0, 10.0)
+    finally:
+        oracle.set_threads(0)
+    variants.append({"value": len(one) * c.Hq / dt1, "unit": UNIT, "cores": 1,
+                     "kind": "oracle, one thread",
+                     "sample": f"{reps1} steps over requests 0..{len(one) - 1}"})
+    res["variants"] = variants
+    return res
 
 
 def main():
@@ -550,6 +745,8 @@ def main():
     ap.add_argument("--plan", action="store_true",
                     help="add the vt_plan_requests launch to the step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-workload rows (configs 1-5) of the default run")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
