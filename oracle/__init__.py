@@ -68,6 +68,9 @@ def _load(kind: str = "f64"):
             lib.vto_select_pages.argtypes = [p, i32, i32, i32, i32, p, i64, p, p, i64, i32, i32,
                                              i32, i32, p, p, p]
             lib.vto_select_pages.restype = ctypes.c_int
+            lib.vto_select_pages_approx.argtypes = [p, i32, i32, i32, i32, p, i64, p, p, i64,
+                                                    i32, i32, i32, i32, ctypes.c_uint64, p, p]
+            lib.vto_select_pages_approx.restype = ctypes.c_int
             lib.vto_sparse_attention.argtypes = [p, i32, i32, i32, i32, i32, p, i64, i64, i64, p,
                                                  i64, i64, i64, i64, i32, p, i64, p, p, p, i32,
                                                  f64, p, p]
@@ -144,6 +147,27 @@ def select_pages(q, page_table, seq_lens, centroids, topk, bos, eos, page_size=1
                                   _ptr(scores) if want_scores else None)
     _check(rc, "select_pages")
     return (sel, n_sel, scores) if want_scores else (sel, n_sel)
+
+
+def select_pages_approx(q, page_table, seq_lens, centroids, topk, bos, eos, seed,
+                        page_size=16):
+    """The lossy indexer mode: one radix pass over the fp32 scores (1024 bins linear between
+    the smallest and largest), every bin above the topk-th score's bin kept, that bin's
+    candidates taken in cyclic order from a SplitMix64-drawn start.  Returns (sel, n_sel)."""
+    B, hq, d = q.shape
+    P, hkv, dc = centroids.shape
+    assert dc == d and q.is_contiguous() and centroids.is_contiguous()
+    page_table, seq_lens = _i32(page_table), _i32(seq_lens)
+    kmax = topk + bos + eos
+    sel = torch.empty((B, hkv, kmax), dtype=torch.int32)
+    n_sel = torch.empty((B, hkv), dtype=torch.int32)
+    rc = _load().vto_select_pages_approx(_ptr(_bits(q)), B, hq, hkv, d, _ptr(page_table),
+                                         page_table.shape[1], _ptr(seq_lens), _ptr(centroids),
+                                         P, page_size, topk, bos, eos,
+                                         ctypes.c_uint64(seed & (2**64 - 1)), _ptr(sel),
+                                         _ptr(n_sel))
+    _check(rc, "select_pages_approx")
+    return sel, n_sel
 
 
 def sparse_attention(q, k_pool, v_pool, page_table, seq_lens, sel, n_sel, sm_scale,

@@ -237,6 +237,131 @@ int vto_select_pages(const uint16_t* q, int32_t batch, int32_t num_q_heads,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Lossy mode of the indexer: an early-terminating ("stochastic radix") top-k. */
+/* ------------------------------------------------------------------------ */
+
+/* SplitMix64's output step (Steele, Lea and Flood, "Fast splittable pseudorandom number
+ * generators", OOPSLA 2014): advance by the golden gamma, then the two xor-shift-multiply
+ * rounds.  The counter-based generator the lossy mode draws its random start from. */
+static uint64_t vto_splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+/*
+ * The indexer's "stochastic radix top-k" (rndamp.com article, "A dual-stage programmable
+ * abstraction": a lossy top-k with early termination, for the indexing stage), read as:
+ * one radix pass over the candidates' scores, then stop.  Per unit with n > kmax:
+ *   - scores s_i as in vto_select_pages, rounded to fp32 (f_i; the kernels decide in fp32);
+ *   - lo, hi = the smallest and largest f_i; if hi > lo (and finite) each candidate gets
+ *     bin_i = min(1023, (int)((f_i - lo) * (1024 / (hi - lo)))), every step in fp32;
+ *     otherwise every candidate is in bin 0;
+ *   - B = the bin holding the topk-th largest score (counting bins from the top);
+ *   - every candidate in a bin above B is kept; instead of refining inside B the pass
+ *     ends there: the remaining need slots go to B's candidates in cyclic order of their
+ *     position c = i - bos, starting at r = splitmix64(seed + b*Hkv + h) mod m.
+ * The reserved pages and the dense rule are those of vto_select_pages.
+ */
+int vto_select_pages_approx(const uint16_t* q, int32_t batch, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim, const int32_t* page_table,
+                            int64_t pt_stride, const int32_t* seq_lens, const float* centroids,
+                            int64_t num_pages, int32_t page_size, int32_t topk, int32_t bos,
+                            int32_t eos, uint64_t seed, int32_t* sel, int32_t* n_sel) {
+  if (batch < 0 || num_q_heads < 1 || num_kv_heads < 1 || head_dim < 1 || page_size < 1 ||
+      pt_stride < 1 || topk < 0 || bos < 0 || eos < 0 || num_q_heads % num_kv_heads != 0)
+    return VTO_ERR_ARG;
+  int rc = check_lengths(seq_lens, batch, page_size, pt_stride);
+  if (rc) return rc;
+  const int32_t G = num_q_heads / num_kv_heads;
+  const int32_t kmax = topk + bos + eos;
+  const int64_t units = (int64_t)batch * num_kv_heads;
+  int bad_page = 0;
+#pragma omp parallel num_threads(vto_get_threads()) reduction(| : bad_page)
+  {
+    vto_real* qm = (vto_real*)malloc(sizeof(vto_real) * (size_t)head_dim);
+    float* f = (float*)malloc(sizeof(float) * (size_t)pt_stride);
+    int32_t* bin = (int32_t*)malloc(sizeof(int32_t) * (size_t)pt_stride);
+    char* keep = (char*)malloc((size_t)pt_stride);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t u = 0; u < units; ++u) {
+      const int32_t b = (int32_t)(u / num_kv_heads);
+      const int32_t h = (int32_t)(u % num_kv_heads);
+      const int32_t n = (int32_t)ceil_div64(seq_lens[b], page_size);
+      int32_t* out = sel + u * kmax;
+      for (int32_t j = 0; j < kmax; ++j) out[j] = -1;
+      if (n <= kmax) {
+        for (int32_t i = 0; i < n; ++i) out[i] = i;
+        n_sel[u] = n;
+        continue;
+      }
+      for (int32_t d = 0; d < head_dim; ++d) {
+        vto_real s = 0.0;
+        for (int32_t j = 0; j < G; ++j)
+          s += bf16_to_f64(q[((int64_t)b * num_q_heads + (int64_t)h * G + j) * head_dim + d]);
+        qm[d] = s / (vto_real)G;
+      }
+      const int32_t m = n - bos - eos;
+      float lo = INFINITY, hi = -INFINITY;
+      for (int32_t c = 0; c < m; ++c) {
+        const int64_t p = page_table[(int64_t)b * pt_stride + bos + c];
+        if (p < 0 || p >= num_pages) {
+          bad_page = 1;
+          f[c] = -INFINITY;
+          continue;
+        }
+        const float* cr = centroids + (p * num_kv_heads + h) * head_dim;
+        vto_real s = 0.0;
+        for (int32_t d = 0; d < head_dim; ++d) s += qm[d] * (vto_real)cr[d];
+        f[c] = (float)s;
+        if (f[c] < lo) lo = f[c];
+        if (f[c] > hi) hi = f[c];
+      }
+      const float width = hi - lo;
+      const int linear = hi > lo && isfinite(width);
+      const float inv = linear ? 1024.0f / width : 0.0f;
+      int32_t count[1024];
+      memset(count, 0, sizeof count);
+      for (int32_t c = 0; c < m; ++c) {
+        int32_t k = 0;
+        if (linear) {
+          const float x = (f[c] - lo) * inv;
+          k = x >= 1023.0f ? 1023 : (int32_t)x;
+        }
+        bin[c] = k;
+        count[k] += 1;
+      }
+      int32_t B = 1023, above = 0;
+      while (B > 0 && above + count[B] < topk) above += count[B--];
+      int32_t need = topk - above;
+      memset(keep, 0, (size_t)n);
+      for (int32_t i = 0; i < bos; ++i) keep[i] = 1;
+      for (int32_t i = n - eos; i < n; ++i) keep[i] = 1;
+      for (int32_t c = 0; c < m; ++c)
+        if (bin[c] > B) keep[bos + c] = 1;
+      const int32_t r = (int32_t)(vto_splitmix64(seed + (uint64_t)u) % (uint64_t)m);
+      for (int32_t t = 0; t < m && need > 0; ++t) {
+        const int32_t c = (r + t) % m;
+        if (bin[c] == B) {
+          keep[bos + c] = 1;
+          --need;
+        }
+      }
+      int32_t cnt = 0;
+      for (int32_t i = 0; i < n; ++i)
+        if (keep[i]) out[cnt++] = i;
+      n_sel[u] = cnt;
+    }
+    free(qm);
+    free(f);
+    free(bin);
+    free(keep);
+  }
+  return bad_page ? VTO_ERR_PAGE : VTO_OK;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Exact softmax attention over the selected pages.                          */
 /* ------------------------------------------------------------------------ */
 

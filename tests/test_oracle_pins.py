@@ -473,3 +473,86 @@ def test_fp32_timing_copy_tracks_the_oracle(oracle):
     assert torch.allclose(c32, c64, rtol=1e-6, atol=1e-7)
     assert torch.equal(n32, n64) and torch.equal(s32, s64)
     assert (o32 - o64).abs().max().item() < 1e-4 and (l32 - l64).abs().max().item() < 1e-4
+
+
+# --------------------------------------------------------------------------------------
+# the lossy indexer mode (one radix pass, early termination, random start in the last bin)
+# --------------------------------------------------------------------------------------
+
+# SplitMix64's published output sequence from state 0 (Steele, Lea and Flood 2014; the
+# reference generator's first three outputs): the start of the cyclic fill for unit 0 with
+# seed = 0, gamma and 2 gamma.
+GAMMA = 0x9E3779B97F4A7C15
+SPLITMIX64_FROM_ZERO = (0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F)
+
+
+def _one_head_case(values, topk, bos=1, eos=1):
+    """One request, Hkv = G = 1, D = 4, q = e0, centroid of page i = (values[i], 0, 0, 0):
+    the score of page i is values[i]."""
+    n = len(values)
+    pt, seq = _identity_batch(n)
+    q = torch.zeros(1, 1, 4)
+    q[0, 0, 0] = 1.0
+    cent = torch.zeros(n, 1, 4)
+    cent[:, 0, 0] = torch.tensor(values, dtype=torch.float32)
+    return q.to(torch.bfloat16), pt, seq, cent
+
+
+def test_approx_equals_exact_when_every_score_has_its_own_bin(oracle):
+    """m <= 1024 candidates with evenly spaced scores: one per bin, so the single pass is exact."""
+    g = torch.Generator().manual_seed(21)
+    m = 300
+    vals = (torch.randperm(m + 2, generator=g).float() * 0.5).tolist()
+    q, pt, seq, cent = _one_head_case(vals, 30)
+    exact = oracle.select_pages(q, pt, seq, cent, 30, 1, 1)
+    for seed in (0, 5, 2 ** 63 + 11):
+        approx = oracle.select_pages_approx(q, pt, seq, cent, 30, 1, 1, seed)
+        assert torch.equal(approx[0], exact[0]) and torch.equal(approx[1], exact[1])
+
+
+@pytest.mark.parametrize("which", [0, 1, 2])
+def test_approx_fill_of_the_last_bin_starts_at_the_published_draw(oracle, which):
+    """Every score equal: all candidates share bin 0, so the pass keeps topk of them in cyclic
+    order from r = splitmix64(seed + unit) mod m; for unit 0 and seed = which * gamma that is
+    the generator's published output number which + 1."""
+    n, topk = 50, 7
+    m = n - 2
+    q, pt, seq, cent = _one_head_case([1.5] * n, topk)
+    seed = (which * GAMMA) % 2 ** 64
+    sel, n_sel = oracle.select_pages_approx(q, pt, seq, cent, topk, 1, 1, seed)
+    r = SPLITMIX64_FROM_ZERO[which] % m
+    want = sorted([0, n - 1] + [1 + (r + t) % m for t in range(topk)])
+    assert int(n_sel[0, 0]) == topk + 2
+    assert sel[0, 0, : topk + 2].tolist() == want
+
+
+def test_approx_keeps_every_page_clear_of_the_boundary_and_is_valid(oracle):
+    """Random batches: the lossy set has the exact size, holds the reserved pages, and keeps
+    every candidate scoring more than two bin widths above the exact k-th score; its recall of
+    the exact top-k stays high."""
+    from paged_block_sparse_vt_b200.workloads import config, make_workload
+    w = make_workload(config(2, B=6, len_lo=2000, len_hi=12000, pool_pages=6000))
+    c = w["config"]
+    full = torch.cat([w["prebuilt_pages"], w["fill_pages"]]).to(torch.int32)
+    cent = torch.zeros((w["P"], c.Hkv, c.D))
+    oracle.build_centroids(w["k_pool"], full, cent)
+    sel, n_sel, scores = oracle.select_pages(w["q"], w["page_table"], w["seq_lens"], cent, c.topk,
+                                             c.bos, c.eos, want_scores=True)
+    asel, an = oracle.select_pages_approx(w["q"], w["page_table"], w["seq_lens"], cent, c.topk,
+                                          c.bos, c.eos, 99)
+    assert torch.equal(an, n_sel)
+    recalls = []
+    for b in range(c.B):
+        n = (int(w["seq_lens"][b]) + 15) // 16
+        for h in range(c.Hkv):
+            got = set(asel[b, h, : an[b, h]].tolist())
+            want = set(sel[b, h, : n_sel[b, h]].tolist())
+            assert {0, n - 1} <= got and len(got) == c.kmax
+            s = scores[b, h, 1:n - 1]
+            kth = min(scores[b, h, i].item() for i in want if 0 < i < n - 1)
+            width = (s.max() - s.min()).item() / 1024
+            for i in range(1, n - 1):
+                if scores[b, h, i].item() > kth + 2 * width:
+                    assert i in got
+            recalls.append(len(got & want) / len(want))
+    assert min(recalls) >= 0.9 and sum(recalls) / len(recalls) >= 0.97
