@@ -142,6 +142,25 @@ vt_status vt_select_pages(const vt_paged_kv* kv, const vt_decode_args* a, int32_
                           int32_t* n_sel, void* stream);
 
 /*
+ * The indexer's lossy mode ("stochastic radix top-k": a lossy, early-terminating top-k for
+ * the indexing stage, rndamp.com article, "A dual-stage programmable abstraction"), as
+ * vt_select_pages with the exact top-k replaced by one radix pass that stops there:
+ *   - the candidates' fp32 scores go into 1024 bins linear between their smallest and
+ *     largest score (IEEE fp32: bin = min(1023, (int)((s - lo) * (1024 / (hi - lo)))), one
+ *     bin when hi == lo);
+ *   - every candidate in a bin above the bin B of the topk-th largest score is kept;
+ *   - B is not refined: its remaining slots go to its candidates in cyclic order of their
+ *     position c = i - bos, starting at splitmix64(seed + b*Hkv + h) mod m (m candidates;
+ *     SplitMix64's output step, Steele, Lea and Flood 2014).
+ * The selected set always has topk candidates plus the reserved pages (same sel / n_sel
+ * layout as vt_select_pages), and every candidate scoring a bin width or more above the
+ * exact topk-th score is in it; pages of the same bin as the topk-th score may differ from
+ * the exact top-k.  Same arguments, errors and status bits as vt_select_pages.
+ */
+vt_status vt_select_pages_approx(const vt_paged_kv* kv, const vt_decode_args* a, uint64_t seed,
+                                 int32_t* sel, int32_t* n_sel, void* stream);
+
+/*
  * Sparse attention over a given selection ("performs the actual attention" on
  * the selected blocks through the paged layout): for each query head hq of
  * request b, exact softmax(sm_scale * q K^T) V over the valid tokens of the
@@ -177,6 +196,25 @@ vt_status vt_sparse_decode(const vt_paged_kv* kv, const vt_decode_args* a, const
 vt_status vt_sparse_decode_fused(const vt_paged_kv* kv, const vt_decode_args* a, void* out,
                                  float* lse, int32_t* sel, int32_t* n_sel, void* workspace,
                                  size_t workspace_bytes, void* stream);
+
+/*
+ * One decode step of one layer in one launch: the cache-side centroid build of the pages
+ * that filled at this step (as vt_build_centroids on fill_pages[0, n_fill)) and
+ * vt_sparse_decode_fused, for a serving loop that runs both every step (README "Using Your
+ * Sparse Attention with SGLang": the engine replays each step as a captured CUDA graph).
+ * The build items run on the same persistent CTAs, ahead of the scans, and are not waited
+ * for: a page filled at this step is its request's last page, which with eos >= 1 is a
+ * reserved page that no score of this step reads.  So n_fill > 0 needs eos >= 1
+ * (VT_ERR_UNSUPPORTED otherwise), `centroids` must be the cache args->centroids points to,
+ * and fill_pages must hold only pages that this step does not score (the last page of their
+ * request); other pages would be read while they are written.  Same workspace, results and
+ * errors as vt_sparse_decode_fused; out-of-range fill_pages entries set VT_DEV_BAD_PAGE.
+ * Where the fused call needs no workspace (B > 2048) the build is its own launch first.
+ */
+vt_status vt_sparse_decode_step(const vt_paged_kv* kv, const vt_decode_args* a,
+                                const int32_t* fill_pages, int32_t n_fill, float* centroids,
+                                void* out, float* lse, int32_t* sel, int32_t* n_sel,
+                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Bytes of workspace vt_sparse_decode_fused needs for these arguments (0 if

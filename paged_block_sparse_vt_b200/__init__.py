@@ -19,12 +19,15 @@ from .binding import (  # noqa: F401
     load_library,
     prepare_build_centroids,
     prepare_sparse_decode_fused,
+    prepare_sparse_decode_step,
     vt_abi_version,
     vt_build_centroids,
     vt_fused_workspace_size,
     vt_plan_requests,
     vt_select_pages,
+    vt_select_pages_approx,
     vt_sparse_decode,
     vt_sparse_decode_fused,
+    vt_sparse_decode_step,
     vt_sparse_decode_fused_static,
 )

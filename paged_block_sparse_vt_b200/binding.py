@@ -50,7 +50,8 @@ class DecodeArgs(ctypes.Structure):
     ]
 
 
-EXPORTS = ("vt_build_centroids", "vt_select_pages", "vt_sparse_decode", "vt_sparse_decode_fused",
+EXPORTS = ("vt_build_centroids", "vt_select_pages", "vt_select_pages_approx",
+           "vt_sparse_decode", "vt_sparse_decode_fused", "vt_sparse_decode_step",
            "vt_fused_workspace_size", "vt_sparse_decode_fused_static", "vt_plan_requests",
            "vt_status_string",
            "vt_last_error_detail", "vt_abi_version")
@@ -76,8 +77,10 @@ def load_library(path: str = LIB_PATH):
             sigs = {
                 "vt_build_centroids": [kv, P, I32, P, P, P],
                 "vt_select_pages": [kv, args, P, P, P],
+                "vt_select_pages_approx": [kv, args, ctypes.c_uint64, P, P, P],
                 "vt_sparse_decode": [kv, args, P, P, P, P, P],
                 "vt_sparse_decode_fused": [kv, args, P, P, P, P, P, ctypes.c_size_t, P],
+                "vt_sparse_decode_step": [kv, args, P, I32, P, P, P, P, P, P, ctypes.c_size_t, P],
                 "vt_sparse_decode_fused_static": [kv, args, P, P, P, P, P],
                 "vt_plan_requests": [P, I32, P, P],
             }
@@ -196,6 +199,26 @@ def vt_select_pages(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bo
     return sel, n_sel
 
 
+def vt_select_pages_approx(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos, eos,
+                           seed, sel=None, n_sel=None, order=None, status=None, head_dim_v=None):
+    """The indexer's lossy mode (one radix pass, seeded start in the last bin).  Returns
+    (sel [B,Hkv,kmax], n_sel [B,Hkv])."""
+    lib = load_library()
+    kv = paged_kv(k_pool, v_pool, head_dim_v)
+    a = decode_args(q, page_table, seq_lens, centroids, topk, bos, eos, 1.0, order, status)
+    kmax = topk + bos + eos
+    B, hkv = q.shape[0], k_pool.shape[2]
+    if sel is None:
+        sel = torch.empty((B, hkv, kmax), dtype=torch.int32, device=q.device)
+    if n_sel is None:
+        n_sel = torch.empty((B, hkv), dtype=torch.int32, device=q.device)
+    rc = lib.vt_select_pages_approx(ctypes.byref(kv), ctypes.byref(a),
+                                    ctypes.c_uint64(int(seed) & (2 ** 64 - 1)), sel.data_ptr(),
+                                    n_sel.data_ptr(), _stream(q))
+    _check(rc, "vt_select_pages_approx")
+    return sel, n_sel
+
+
 def vt_sparse_decode(q, k_pool, v_pool, page_table, seq_lens, sel, n_sel, sm_scale, out=None,
                      lse=None, status=None, head_dim_v=None, want_lse=True):
     """Attention over a given page selection.  Returns (out [B,Hq,Dv] bf16, lse [B,Hq] or None)."""
@@ -260,6 +283,35 @@ def vt_sparse_decode_fused(q, k_pool, v_pool, page_table, seq_lens, centroids, t
                                     _ptr(sel), _ptr(n_sel), _ptr(workspace),
                                     0 if workspace is None else workspace.numel(), _stream(q))
     _check(rc, "vt_sparse_decode_fused")
+    return out, lse, sel, n_sel
+
+
+def vt_sparse_decode_step(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos, eos,
+                          sm_scale, fill_pages, out=None, lse=None, sel=None, n_sel=None,
+                          order=None, status=None, head_dim_v=None, want_lse=True,
+                          workspace=None):
+    """One step in one launch: the centroid build of fill_pages (int32, the pages filled at this
+    step; written into ``centroids``) and the fused selection + attention.  Returns
+    (out, lse, sel, n_sel)."""
+    lib = load_library()
+    kv = paged_kv(k_pool, v_pool, head_dim_v)
+    a = decode_args(q, page_table, seq_lens, centroids, topk, bos, eos, sm_scale, order, status)
+    _need(fill_pages, "fill_pages", torch.int32, contiguous=True)
+    B, hq = q.shape[0], q.shape[1]
+    if out is None:
+        out = torch.empty((B, hq, kv.head_dim_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = int(lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(a)))
+        workspace = torch.zeros(n, dtype=torch.uint8, device=q.device) if n else None
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8, contiguous=True)
+    rc = lib.vt_sparse_decode_step(ctypes.byref(kv), ctypes.byref(a), fill_pages.data_ptr(),
+                                   fill_pages.numel(), centroids.data_ptr(), out.data_ptr(),
+                                   _ptr(lse), _ptr(sel), _ptr(n_sel), _ptr(workspace),
+                                   0 if workspace is None else workspace.numel(), _stream(q))
+    _check(rc, "vt_sparse_decode_step")
     return out, lse, sel, n_sel
 
 
@@ -368,6 +420,25 @@ def prepare_sparse_decode_fused(q, k_pool, v_pool, page_table, seq_lens, centroi
             order, status, workspace)
     return PreparedCall(lib.vt_sparse_decode_fused, args, q.get_device(), "vt_sparse_decode_fused",
                         keep, (out, lse, sel, n_sel))
+
+
+def prepare_sparse_decode_step(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos,
+                               eos, sm_scale, fill_pages, out, lse=None, sel=None, n_sel=None,
+                               order=None, status=None, head_dim_v=None,
+                               workspace=None) -> PreparedCall:
+    """vt_sparse_decode_step bound to these tensors (``fill_pages`` included: its contents may
+    change between runs, its length may not); ``run()`` returns (out, lse, sel, n_sel)."""
+    lib = load_library()
+    fused = prepare_sparse_decode_fused(q, k_pool, v_pool, page_table, seq_lens, centroids, topk,
+                                        bos, eos, sm_scale, out, lse, sel, n_sel, order, status,
+                                        head_dim_v, workspace)
+    _need(fill_pages, "fill_pages", torch.int32, contiguous=True)
+    kv_ref, a_ref = fused._args[0], fused._args[1]
+    P = ctypes.c_void_p
+    args = (kv_ref, a_ref, P(fill_pages.data_ptr()), ctypes.c_int32(fill_pages.numel()),
+            P(centroids.data_ptr())) + fused._args[2:]
+    return PreparedCall(lib.vt_sparse_decode_step, args, q.get_device(), "vt_sparse_decode_step",
+                        fused._keep + (fill_pages,), fused.result)
 
 
 def vt_abi_version() -> int:

@@ -203,7 +203,10 @@ size_t persist_bytes(const Shape& sh, const DecodeParams& p, int64_t unit_cap) {
 // unit_cap: units the persistent path's counter arrays are laid out for (0: exactly B * Hkv)
 vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int mode,
                             int32_t* sel, int32_t* n_sel, void* out, float* lse, void* ws,
-                            size_t ws_bytes, void* stream, int64_t unit_cap = 0) {
+                            size_t ws_bytes, void* stream, int64_t unit_cap = 0,
+                            bool approx = false, uint64_t seed = 0,
+                            const int32_t* fill_pages = nullptr, int n_fill = 0,
+                            float* cent_out = nullptr) {
   Shape sh;
   DecodeParams p;
   vt_status s = fill_params(kv, a, mode != kDecode, &sh, &p);
@@ -213,12 +216,30 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
   if (mode == kDecode && (!sel || !n_sel)) return fail(VT_ERR_INVALID_ARG, "sel/n_sel is NULL");
   if (mode == kFused && ((sel == nullptr) != (n_sel == nullptr)))
     return fail(VT_ERR_INVALID_ARG, "sel and n_sel must both be given or both be NULL");
-  if (a->batch == 0) return ok();
+  if (a->batch == 0) {
+    if (n_fill > 0) {
+      cudaError_t e = launch_build_centroids(*kv, fill_pages, n_fill, cent_out, a->status,
+                                             static_cast<cudaStream_t>(stream));
+      if (e != cudaSuccess) return cuda_fail(e, "build_centroids launch");
+    }
+    return ok();
+  }
   p.sel = sel;
   p.n_sel = n_sel;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
+  p.approx = approx ? 1 : 0;
+  p.seed = seed;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_fill > 0 && !(mode == kFused && use_persistent(sh, a))) {
+    // no persistent launch to fold the build into: it runs first, as its own launch
+    cudaError_t e = launch_build_centroids(*kv, fill_pages, n_fill, cent_out, a->status, st);
+    if (e != cudaSuccess) return cuda_fail(e, "build_centroids launch");
+    n_fill = 0;
+  }
+  p.fill_pages = fill_pages;
+  p.n_fill = n_fill;
+  p.cent_out = cent_out;
   if (mode == kFused && use_persistent(sh, a)) {
     const size_t need = persist_bytes(sh, p, unit_cap);
     if (!ws || ws_bytes < need)
@@ -304,6 +325,12 @@ vt_status vt_select_pages(const vt_paged_kv* kv, const vt_decode_args* a, int32_
   return launch_query_side(kv, a, kSelect, sel, n_sel, nullptr, nullptr, nullptr, 0, stream);
 }
 
+vt_status vt_select_pages_approx(const vt_paged_kv* kv, const vt_decode_args* a, uint64_t seed,
+                                 int32_t* sel, int32_t* n_sel, void* stream) {
+  return launch_query_side(kv, a, kSelect, sel, n_sel, nullptr, nullptr, nullptr, 0, stream, 0,
+                           true, seed);
+}
+
 vt_status vt_sparse_decode(const vt_paged_kv* kv, const vt_decode_args* a, const int32_t* sel,
                            const int32_t* n_sel, void* out, float* lse, void* stream) {
   return launch_query_side(kv, a, kDecode, const_cast<int32_t*>(sel),
@@ -357,6 +384,24 @@ vt_status vt_sparse_decode_fused_static(const vt_paged_kv* kv, const vt_decode_a
   }
   return launch_query_side(kv, a, kFused, sel, n_sel, out, lse, ws, ws_bytes, stream,
                            kStaticUnitCap);
+}
+
+vt_status vt_sparse_decode_step(const vt_paged_kv* kv, const vt_decode_args* a,
+                                const int32_t* fill_pages, int32_t n_fill, float* centroids,
+                                void* out, float* lse, int32_t* sel, int32_t* n_sel,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (n_fill < 0) return fail(VT_ERR_INVALID_ARG, "n_fill < 0");
+  if (n_fill > 0) {
+    if (!fill_pages || !centroids) return fail(VT_ERR_INVALID_ARG, "fill_pages/centroids is NULL");
+    if (!a || centroids != a->centroids)
+      return fail(VT_ERR_INVALID_ARG, "centroids must be the cache args->centroids points to");
+    if (a->eos < 1)
+      return fail(VT_ERR_UNSUPPORTED,
+                  "filled pages are built beside the scans: needs eos >= 1 (the last page is "
+                  "then never scored)");
+  }
+  return launch_query_side(kv, a, kFused, sel, n_sel, out, lse, workspace, workspace_bytes,
+                           stream, 0, false, 0, fill_pages, n_fill, centroids);
 }
 
 vt_status vt_plan_requests(const int32_t* seq_lens, int32_t batch, int32_t* order, void* stream) {

@@ -6,11 +6,9 @@
 // centroid per page.
 //
 // Pure HBM stream: each thread owns 8 consecutive dims (one 16-byte load per token) of one
-// (page, KV head) and issues all 16 token loads before using them.  Consecutive threads
-// cover consecutive 16-byte chunks, so a warp reads whole 256-byte head rows.  The sum is
-// accumulated in fp64, where 16 bf16 values add exactly for any realistic exponent spread,
-// so the fp32 centroid is the exact mean rounded once -- independent of summation order.
-#include "common.cuh"
+// (page, KV head) (build_centroid_chunk).  Consecutive threads cover consecutive 16-byte
+// chunks, so a warp reads whole 256-byte head rows.
+#include "centroid_chunk.cuh"
 
 namespace vt {
 
@@ -36,26 +34,7 @@ __global__ void __launch_bounds__(256) build_centroids_kernel(
     if (rem == 0) flag(status, VT_DEV_BAD_PAGE);
     return;
   }
-  const __nv_bfloat16* base = k_pool + p * sk_p + (int64_t)h * sk_h + (int64_t)c * 8;
-  uint4 r[kPage];
-#pragma unroll
-  for (int t = 0; t < kPage; ++t) r[t] = ld_stream_u4(base + (int64_t)t * sk_t);
-  double acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
-#pragma unroll
-  for (int t = 0; t < kPage; ++t) {
-    float f[8];
-    unpack8(r[t], f);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] += (double)f[i];
-  }
-  float o[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) o[i] = __double2float_rn(acc[i] * (1.0 / kPage));
-  float4* dst = reinterpret_cast<float4*>(centroids + (p * num_kv_heads + h) * head_dim + c * 8);
-  dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-  dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+  build_centroid_chunk(k_pool, p, h, c, sk_p, sk_t, sk_h, num_kv_heads, head_dim, centroids);
 }
 
 cudaError_t launch_build_centroids(const vt_paged_kv& kv, const int32_t* pages, int n_pages,

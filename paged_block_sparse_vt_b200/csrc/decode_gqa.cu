@@ -242,9 +242,15 @@ __global__ void __launch_bounds__(kGqaThreads) gqa_decode_kernel(const DecodePar
     for (int j = tid; j < p.eos; j += NT) s_sel[p.bos + p.topk + j] = n - p.eos + j;
     __syncthreads();
     const int bos = p.bos, topk = p.topk;
-    block_topk<NT>(s_key, m, topk, s_hist, s_small, [&](int j, int pos) {
+    auto put = [&](int j, int pos) {
       if (pos < topk) s_sel[bos + pos] = bos + j;  // exactly topk are emitted; guard anyway
-    });
+    };
+    if (p.approx) {
+      const int start = (int)(splitmix64(p.seed + (uint64_t)unit) % (uint64_t)m);
+      approx_topk<NT>(s_key, m, topk, start, s_hist, s_small, put);
+    } else {
+      block_topk<NT>(s_key, m, topk, s_hist, s_small, put);
+    }
   }
   if (MODE != kDecode && rank == 0 && p.sel) {
     for (int j = tid; j < p.kmax; j += NT)

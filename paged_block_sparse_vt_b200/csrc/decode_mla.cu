@@ -238,9 +238,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const Decode
         for (int j = tid; j < p.eos; j += NT) s_sel[p.bos + p.topk + j] = n - p.eos + j;
         __syncthreads();
         const int bos = p.bos, topk = p.topk;
-        block_topk<NT>(s_key, m, topk, s_hist, s_small, [&](int j, int pos) {
+        auto put = [&](int j, int pos) {
           if (pos < topk) s_sel[bos + pos] = bos + j;  // exactly topk are emitted
-        });
+        };
+        if (p.approx) {
+          const int start = (int)(splitmix64(p.seed + (uint64_t)unit) % (uint64_t)m);
+          approx_topk<NT>(s_key, m, topk, start, s_hist, s_small, put);
+        } else {
+          block_topk<NT>(s_key, m, topk, s_hist, s_small, put);
+        }
       }
       cluster.sync();  // #2
       // Only the attending modes need the selection in every CTA.  In kSelect mode rank 0

@@ -26,6 +26,14 @@ struct DecodeParams {
   float qscale;  // sm_scale * log2(e): scores are kept in base-2 units
   const int32_t* order;
   int32_t* status;
+  // the fused step's centroid build of the pages filled at this step (before its scans;
+  // never pages that this step scores): page ids, their count, the centroid cache written
+  const int32_t* fill_pages;
+  int n_fill;
+  float* cent_out;
+  // the indexer's lossy mode (select only): one radix pass, a seeded start in the last bin
+  int approx;
+  unsigned long long seed;
   // selection: written by kSelect / kFused (may be null in kFused), read by kDecode
   int32_t* sel;
   int32_t* n_sel;

@@ -23,6 +23,7 @@
 //                   with several pieces, the last one waits for the others' partials in the
 //                   workspace and merges them in registers.
 // Queue, claims and counters work as in the GQA persistent kernel (fused_persistent.cu).
+#include "centroid_chunk.cuh"
 #include "decode_params.cuh"
 #include "topk.cuh"
 
@@ -207,7 +208,8 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
   uint32_t qbase = 0;  // thread 0: the claim count when this launch began
-  auto claim = [&]() { return (int)(atomicAdd(w.ctr + 0, 1u) - qbase); };
+  // items are numbered from -n_fill: the build items of the pages filled at this step first
+  auto claim = [&]() { return (int)(atomicAdd(w.ctr + 0, 1u) - qbase) - p.n_fill; };
 
   // ---- schedule: exclusive prefix of scan items over the requests
   {
@@ -263,10 +265,26 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
     __syncthreads();
     if (t >= total_items) {
       if (tid == 0 && t == total_items + (int)gridDim.x - 1)
-        w.ctr[1] = qbase + (uint32_t)total_items + gridDim.x;
+        w.ctr[1] = qbase + (uint32_t)(p.n_fill + total_items) + gridDim.x;
       break;
     }
     int next = -1;
+    if (t < 0) {
+      // ---------------------------------------------------------------- build item
+      // the centroid of one page filled at this step, which no score of this step reads (the
+      // page is its request's reserved last page)
+      const int64_t pg = p.fill_pages[t + p.n_fill];
+      if (pg < 0 || pg >= p.num_pages) {
+        if (tid == 0) flag(p.status, VT_DEV_BAD_PAGE);
+      } else {
+        for (int idx = tid; idx < D / 8; idx += NT)
+          build_centroid_chunk(p.k_pool, pg, 0, idx, p.sk_p, p.sk_t, p.sk_h, 1, D, p.cent_out);
+      }
+      __syncthreads();
+      if (tid == 0) s_misc[0] = claim();
+      __syncthreads();
+      continue;
+    }
 
     // decode the item: (scan, request, chunk) or (attention, request, piece)
     bool is_scan = false;

@@ -27,7 +27,7 @@
 //   items           CTA waits until all of the unit's chunks are counted (every chunk was
 //                   claimed before this item and scan items never wait, so the wait ends),
 //                   merges the candidates with the same exact top-k, attends the pages of its
-//                   piece on the tensor cores (four per warp through a two-slot ring) and
+//                   piece on the tensor cores (eight per warp through a kAttSlots-slot ring) and
 //                   stores a partial (max, sum, acc); the piece that is counted last for
 //                   its unit merges the partials and writes the bf16 output and the lse.
 // The schedule (scan items per request and their prefix) is computed by every CTA from the
@@ -35,6 +35,7 @@
 // the CTA that last uses them and the claim counter runs on across launches (each launch
 // numbers its items from where the previous one stopped), so the workspace needs
 // zero-filling only once and no CTA waits for the others on its way out.
+#include "centroid_chunk.cuh"
 #include "decode_params.cuh"
 #include "gqa_attend.cuh"
 #include "topk.cuh"
@@ -47,6 +48,7 @@ constexpr int kChunk = 256;      // candidate pages per scan item (64 per warp)
 constexpr int kScanRing = 4;     // 8-row centroid batches per warp ring (3 landing)
 constexpr int kPiecePages = 32;  // most selected pages per attention item (8 per warp)
 constexpr int kTailPiecePages = 16;  // the same for the units attended last
+constexpr int kAttSlots = 2;     // page slots per warp's attention ring (kAttSlots - 1 landing)
 constexpr int kMaxPlanB = 2048;  // requests the persistent path takes (schedule kept in smem)
 constexpr int kPersistMinCtas = 3;  // CTAs per SM the registers must allow (<= 168 per thread)
 
@@ -181,7 +183,7 @@ __host__ __device__ inline PersistSmem persist_smem_layout(int D, int G, int B,
   // scan rings, plus the chunk top-k scratch where it does not fit in one ring slot
   const int scan = kPersistWarps * kScanRing * 8 * D * 4 +
                    (8 * D * 4 >= SmallTopk<kPersistThreads>::BYTES ? 0 : SmallTopk<kPersistThreads>::BYTES);
-  const int att = kPersistWarps * 2 * 2 * kPage * (D + 8) * 2;
+  const int att = kPersistWarps * kAttSlots * 2 * kPage * (D + 8) * 2;
   // merge of up to 2 NT candidates: keys, logical and physical pages, small_topk scratch;
   // of more: keys, offsets, block_topk scratch
   const int merge_small = 3 * 2 * kPersistThreads * 4 + SmallTopk<kPersistThreads>::BYTES;
@@ -230,7 +232,8 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
   uint32_t qbase = 0;  // thread 0: the claim count when this launch began
-  auto claim = [&]() { return (int)(atomicAdd(w.ctr + 0, 1u) - qbase); };
+  // items are numbered from -n_fill: the build items of the pages filled at this step first
+  auto claim = [&]() { return (int)(atomicAdd(w.ctr + 0, 1u) - qbase) - p.n_fill; };
 
   // ---- schedule: exclusive prefix of scan items over the requests, in request order
   {
@@ -373,16 +376,29 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
     __syncthreads();  // every thread has read the item before the next claim is stored
     if (t >= total_items) {
       // Every CTA makes one claim per item plus one that ends it, so the launch's claims are
-      // numbered 0 .. total_items + gridDim.x - 1.  The CTA holding the last one knows that
-      // every CTA has read qbase, and sets it for the next launch.
+      // numbered -n_fill .. total_items + gridDim.x - 1.  The CTA holding the last one knows
+      // that every CTA has read qbase, and sets it for the next launch.
       if (tid == 0 && t == total_items + (int)gridDim.x - 1)
-        w.ctr[1] = qbase + (uint32_t)total_items + gridDim.x;
+        w.ctr[1] = qbase + (uint32_t)(p.n_fill + total_items) + gridDim.x;
       break;
     }
     // the next item, claimed by thread 0 once this item's streaming is done (or at its end)
     int next = -1;
 
-    if (t < scan_items) {
+    if (t < 0) {
+      // ---------------------------------------------------------------- build item
+      // the centroids of one page filled at this step (every KV head), which no score of
+      // this step reads: the page is its request's reserved last page
+      const int64_t pg = p.fill_pages[t + p.n_fill];
+      if (pg < 0 || pg >= p.num_pages) {
+        if (tid == 0) flag(p.status, VT_DEV_BAD_PAGE);
+      } else {
+        for (int idx = tid; idx < p.Hkv * (D / 8); idx += NT)
+          build_centroid_chunk(p.k_pool, pg, idx / (D / 8), idx % (D / 8), p.sk_p, p.sk_t,
+                               p.sk_h, p.Hkv, D, p.cent_out);
+      }
+      if (tid == 0) next = claim();
+    } else if (t < scan_items) {
       // ---------------------------------------------------------------- scan item
       const ScanItem it = scan_item(t);
       if (!prepared) {
@@ -654,9 +670,9 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
           if (tid < np) s_phys[tid] = checked(ptrow[s_sel[tid]]);
           __syncthreads();
         }
-        // ---- warp w: pages w + NW i (i < 4) of the piece through a two-slot ring
+        // ---- warp w: pages w + NW i of the piece through a kAttSlots-slot ring
         const int last_valid = L - kPage * (n - 1);
-        const uint32_t ring = region_u32 + warp * 2 * S::SLOT;
+        const uint32_t ring = region_u32 + warp * kAttSlots * S::SLOT;
         auto rows_of = [&](int j) {
           return s_phys[j] < 0 ? 0 : (s_sel[j] == n - 1 ? last_valid : kPage);
         };
@@ -665,21 +681,22 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
           if (i < npw) {
             const int j = warp + NW * i;
             const int64_t pg = s_phys[j] < 0 ? 0 : s_phys[j];
-            stage_page<D>(ring + (i & 1) * S::SLOT, p.k_pool + pg * p.sk_p + (int64_t)h * p.sk_h,
+            stage_page<D>(ring + (i % kAttSlots) * S::SLOT, p.k_pool + pg * p.sk_p + (int64_t)h * p.sk_h,
                           p.v_pool + pg * p.sv_p + (int64_t)h * p.sv_h, p.sk_t, p.sv_t,
                           rows_of(j), p.k_pool, lane);
           }
           cp_async_commit();
         };
-        issue(0);
+#pragma unroll
+        for (int i = 0; i < kAttSlots - 1; ++i) issue(i);
         WarpAttention<D, G> att;
         const int64_t orow = (int64_t)b * p.Hq + (int64_t)h * G;
         att.init(p.q + orow * D, lane);
         for (int i = 0; i < npw; ++i) {
-          issue(i + 1);
-          cp_async_wait<1>();
+          issue(i + kAttSlots - 1);
+          cp_async_wait<kAttSlots - 1>();
           __syncwarp();
-          att.page(ring + (i & 1) * S::SLOT, rows_of(warp + NW * i), p.qscale);
+          att.page(ring + (i % kAttSlots) * S::SLOT, rows_of(warp + NW * i), p.qscale);
           __syncwarp();
         }
         cp_async_wait<0>();

@@ -234,6 +234,158 @@ __device__ void block_topk(const uint32_t* keys, int m, int k, int* hist, int* s
   __syncthreads();
 }
 
+// ---- the lossy mode: one radix pass, then stop --------------------------------------------
+// The indexer's early-terminating ("stochastic radix") top-k of the rndamp.com article, "A
+// dual-stage programmable abstraction", read as: one histogram pass of 1024 bins linear in
+// the fp32 score between the smallest and the largest key (IEEE fp32 steps: (s - lo) * (1024 /
+// (hi - lo)), truncated, capped at 1023; one bin when hi == lo or the range is not finite),
+// every key in a bin above the k-th key's bin B selected, and no refinement inside B: its
+// remaining slots go to B's keys in cyclic index order starting at index `start`.
+
+// SplitMix64's output step (Steele, Lea and Flood 2014): advance by the golden gamma, then
+// two xor-shift-multiply rounds.  The counter-based generator of the lossy mode's start.
+__host__ __device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Scratch in shared memory: hist[kTopkBins] ints, small[64] ints.  Emits exactly k indices
+// (k < m) in ascending order with their positions.
+template <int NT, typename Emit>
+__device__ void approx_topk(const uint32_t* keys, int m, int k, int start, int* hist, int* small,
+                            Emit emit) {
+  constexpr int NW = NT / 32;
+  static_assert(NW <= 8, "small[] holds per-warp counts of at most 8 warps");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (k <= 0) return;
+  if (k >= m) {
+    for (int j = tid; j < m; j += NT) emit(j, j);
+    __syncthreads();
+    return;
+  }
+  uint32_t lo = 0xffffffffu, hi = 0u;
+  for (int j = tid; j < m; j += NT) {
+    const uint32_t key = keys[j];
+    lo = min(lo, key);
+    hi = max(hi, key);
+  }
+  lo = __reduce_min_sync(kFull, lo);
+  hi = __reduce_max_sync(kFull, hi);
+  if (lane == 0) {
+    small[warp] = (int)lo;
+    small[NW + warp] = (int)hi;
+  }
+  for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0;
+  __syncthreads();
+  lo = 0xffffffffu;
+  hi = 0u;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    lo = min(lo, (uint32_t)small[w]);
+    hi = max(hi, (uint32_t)small[NW + w]);
+  }
+  const float flo = key_score(lo), width = __fsub_rn(key_score(hi), flo);
+  const bool linear = width > 0.0f && isfinite(width);
+  const float inv = linear ? __fdiv_rn((float)kTopkBins, width) : 0.0f;
+  auto bin_of = [&](uint32_t key) {
+    if (!linear) return 0;
+    const float x = __fmul_rn(__fsub_rn(key_score(key), flo), inv);
+    return x >= (float)(kTopkBins - 1) ? kTopkBins - 1 : (int)x;
+  };
+  for (int j = tid; j < m; j += NT) atomicAdd(&hist[bin_of(keys[j])], 1);
+  __syncthreads();
+  if (warp == 0) {  // the bin of the k-th largest key (32 bins per lane, top bins in lane 31)
+    constexpr int BPL = kTopkBins / 32;
+    int tot = 0;
+#pragma unroll
+    for (int i = 0; i < BPL; ++i) tot += hist[lane * BPL + ((i + lane) & (BPL - 1))];
+    int incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_down_sync(kFull, incl, o);
+      if (lane + o < 32) incl += y;
+    }
+    const int above_lane = incl - tot;
+    if (above_lane < k && k <= incl) {
+      int acc = above_lane;
+      for (int i = BPL - 1; i >= 0; --i) {
+        const int c = hist[lane * BPL + i];
+        if (acc + c >= k) {
+          small[40] = lane * BPL + i;
+          small[41] = acc;
+          break;
+        }
+        acc += c;
+      }
+    }
+  }
+  __syncthreads();
+  const int B = small[40];
+  const int need = k - small[41];
+  // emit in ascending index order: every warp walks a contiguous range in chunks of 32; the
+  // members of B are ranked in cyclic order from `start`
+  const int R = ((m + NW * 32 - 1) / (NW * 32)) * 32;
+  const int w0 = min(m, warp * R), w1 = min(m, w0 + R);
+  const unsigned lt = (1u << lane) - 1u;
+  int c2 = 0, c1 = 0, c1lo = 0;  // above B; in B; in B with index < start
+  for (int j0 = w0; j0 < w1; j0 += 32) {
+    const int j = j0 + lane;
+    const int b = j < w1 ? bin_of(keys[j]) : -1;
+    c2 += __popc(__ballot_sync(kFull, b > B));
+    c1 += __popc(__ballot_sync(kFull, b == B));
+    c1lo += __popc(__ballot_sync(kFull, b == B && j < start));
+  }
+  __syncthreads();  // everyone is done with small[] reads above
+  if (lane == 0) {
+    small[48 + warp] = c2;
+    small[56 + warp] = c1;
+    small[32 + warp] = c1lo;
+  }
+  __syncthreads();
+  int T1 = 0, L1 = 0, pre2 = 0, pre1 = 0;
+  for (int w = 0; w < NW; ++w) {
+    T1 += small[56 + w];
+    L1 += small[32 + w];
+    if (w < warp) {
+      pre2 += small[48 + w];
+      pre1 += small[56 + w];
+    }
+  }
+  auto taken_tie = [&](int j, int rank_from_0) {  // rank_from_0: members of B below j
+    const int cyc = j >= start ? rank_from_0 - L1 : (T1 - L1) + rank_from_0;
+    return cyc < need;
+  };
+  // offsets of this warp's first selected key: every selected key of earlier warps
+  int sel_off = pre2;
+  {
+    // members of B taken among indices < w0: count them from the prefix counts
+    // (taken(j) depends only on j's rank among B's members, so count ranks [0, pre1))
+    int t = 0;
+    // ranks r < pre1 belong to indices < w0; those with index >= start are the ranks >= L1
+    const int lo_taken = min(pre1, L1);           // ranks [0, lo_taken): index < start
+    // index < start: cyclic rank (T1 - L1) + r, taken when < need
+    t += max(0, min(lo_taken, need - (T1 - L1)));
+    // index >= start: ranks [L1, pre1): cyclic rank r - L1, taken when < need
+    if (pre1 > L1) t += max(0, min(pre1, L1 + need) - L1);
+    sel_off += t;
+  }
+  int rank1 = pre1;
+  for (int j0 = w0; j0 < w1; j0 += 32) {
+    const int j = j0 + lane;
+    const int b = j < w1 ? bin_of(keys[j]) : -1;
+    const unsigned tb = __ballot_sync(kFull, b == B);
+    const int r1 = rank1 + __popc(tb & lt);
+    const bool take = (b > B) || (b == B && taken_tie(j, r1));
+    const unsigned sb = __ballot_sync(kFull, take);
+    if (take) emit(j, sel_off + __popc(sb & lt));
+    sel_off += __popc(sb);
+    rank1 += __popc(tb);
+  }
+  __syncthreads();
+}
+
 // Shared-memory scratch of small_topk (16-byte aligned): hist[HIST] ints that are ZERO on
 // entry (hist[kSmallBins] counts the members of the threshold bin), list[2 NT] (key, index)
 // pairs, cnt[2 NW] ints.
