@@ -122,6 +122,7 @@ def read_peak_hbm():
 
 # the files the timed fused kernel is compiled from
 FUSED_KERNEL_SOURCES = ("fused_persistent.cu", "gqa_attend.cuh", "topk.cuh", "common.cuh",
+                        "centroid_chunk.cuh",
                         "decode_params.cuh")
 
 
@@ -399,10 +400,19 @@ def run_ours(args, world, rank, local):
                                   order=d["order"] if args.plan else None, status=d["status"],
                                   workspace=d["ws"], head_dim_v=c.Dv)
 
-    # A page that fills at this step is its request's reserved last page (eos >= 1) until the
-    # next step, so no score of this step reads its centroid: its build runs on a second
-    # stream beside this step's fused call, and the stream joins again before the next step.
-    side = torch.cuda.Stream(dev) if c.eos >= 1 else None
+    def one_launch(d):  # the build of this step's filled pages and the fused call, one launch
+        vt.vt_sparse_decode_step(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                 d["seq_lens"], d["cent"], c.topk, c.bos, c.eos, c.sm_scale,
+                                 d["fill_pages"], out=d["out"], lse=d["lse"],
+                                 order=d["order"] if args.plan else None, status=d["status"],
+                                 workspace=d["ws"], head_dim_v=c.Dv)
+
+    one = args.step_mode == "one-launch" and c.eos >= 1
+    # Two-call mode: a page that fills at this step is its request's reserved last page
+    # (eos >= 1) until the next step, so no score of this step reads its centroid: its build
+    # runs on a second stream beside this step's fused call, and the stream joins again before
+    # the next step.  One-launch mode folds the same build into the fused launch.
+    side = torch.cuda.Stream(dev) if (c.eos >= 1 and not one) else None
 
     def build_call(d, prepared=False):
         if prepared:
@@ -411,6 +421,16 @@ def run_ours(args, world, rank, local):
             vt.vt_build_centroids(d["k_pool"], d["fill_pages"], d["cent"], status=d["status"])
 
     def step(d, prepared=False, after_fused=None, overlap=True):
+        if one:
+            if args.plan:
+                vt.vt_plan_requests(d["seq_lens"], d["order"])
+            if prepared:
+                d["p_step"].run()
+            else:
+                one_launch(d)
+            if after_fused is not None:
+                after_fused(d)
+            return
         main = torch.cuda.current_stream(dev)
         if side is not None and overlap:
             side.wait_stream(main)  # this step's inputs are in place
@@ -429,7 +449,8 @@ def run_ours(args, world, rank, local):
         if side is not None and overlap:
             main.wait_stream(side)  # the build is done before anything later on this stream
 
-    launches_per_step = 2 + (1 if args.plan else 0)
+    launches_per_step = (1 if one else 2) + (1 if args.plan else 0)
+    dominant = one_launch if one else fused  # the kernel the roofline is about
     for i in range(args.warmup):
         step(reps[i % args.replicas])
     torch.cuda.synchronize(dev)
@@ -443,7 +464,7 @@ def run_ours(args, world, rank, local):
     fused_graph = torch.cuda.CUDAGraph()  # the dominant kernel alone, the same sequence
     with torch.cuda.graph(fused_graph):
         for i in range(args.steps):
-            fused(reps[i % args.replicas])
+            dominant(reps[i % args.replicas])
     torch.cuda.synchronize(dev)
     graph.replay()  # untimed: the first replay of a graph uploads it
     fused_graph.replay()
@@ -482,6 +503,11 @@ def run_ours(args, world, rank, local):
     # eager launches through the public API (no graph): each replica's two calls prepared
     # once (arguments checked and marshalled), as a serving loop does for its fixed buffers
     for d in reps:
+        d["p_step"] = vt.prepare_sparse_decode_step(
+            d["q"], d["k_pool"], d["v_pool"], d["page_table"], d["seq_lens"], d["cent"], c.topk,
+            c.bos, c.eos, c.sm_scale, d["fill_pages"], out=d["out"], lse=d["lse"],
+            order=d["order"] if args.plan else None, status=d["status"], head_dim_v=c.Dv,
+            workspace=d["ws"])
         d["p_build"] = vt.prepare_build_centroids(d["k_pool"], d["fill_pages"], d["cent"],
                                                   status=d["status"])
         d["p_fused"] = vt.prepare_sparse_decode_fused(
@@ -535,7 +561,8 @@ def run_ours(args, world, rank, local):
     ms = elapsed / args.steps * 1e3
     units = c.B * c.Hq
     value = aggregate_value(world, units, args.steps, elapsed)
-    achieved = nbytes["fused"] / (fused_ms / 1e3) / 1e9
+    launch_bytes = nbytes["total"] if one else nbytes["fused"]
+    achieved = launch_bytes / (fused_ms / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -548,8 +575,9 @@ def run_ours(args, world, rank, local):
                           "frac_nominal_8000 against the nominal ~8 TB/s HBM3e figure"),
             "traffic": recorded_traffic(args.config),
             "kernel": ("persist_mla_kernel" if c.mla else "persist_fused_kernel")
-                      + " (vt_sparse_decode_fused)",
-            "algorithmic_bytes_per_launch": nbytes["fused"], "kernel_ms": fused_ms,
+                      + (" (vt_sparse_decode_step: filled pages' build + select + attend)"
+                         if one else " (vt_sparse_decode_fused)"),
+            "algorithmic_bytes_per_launch": launch_bytes, "kernel_ms": fused_ms,
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
             else "fallback 6650 GB/s",
         },
@@ -557,7 +585,9 @@ def run_ours(args, world, rank, local):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "timing": "the K steps as one CUDA graph replayed once, CUDA events on the launching stream",
-        "step": ("vt_build_centroids (pages filled this step) on a second stream beside "
+        "step": ("vt_sparse_decode_step: the centroid build of the pages filled this step "
+                 "and the fused select + attend in one launch" if one else
+                 "vt_build_centroids (pages filled this step) on a second stream beside "
                  "vt_sparse_decode_fused, joined before the next step (e2e: one stream)"
                  if side is not None else "vt_build_centroids then vt_sparse_decode_fused"),
         "clocks": clk,
@@ -639,6 +669,12 @@ def measure_config(vt, cfg: int, dev, peak: float, iters: int = 10) -> dict:
                                           sel=d["sel"], n_sel=d["n_sel"], status=d["status"],
                                           head_dim_v=c.Dv)
 
+    def select_lossy(d):
+        return lambda: vt.vt_select_pages_approx(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                                 d["seq_lens"], d["cent"], c.topk, c.bos, c.eos,
+                                                 0x5EED, sel=d["sel"], n_sel=d["n_sel"],
+                                                 status=d["status"], head_dim_v=c.Dv)
+
     def decode(d):
         return lambda: vt.vt_sparse_decode(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
                                            d["seq_lens"], d["sel"], d["n_sel"], c.sm_scale,
@@ -655,8 +691,11 @@ def measure_config(vt, cfg: int, dev, peak: float, iters: int = 10) -> dict:
                        f"{lengths_text(c)}, top-{c.topk}+{c.bos}+{c.eos}, pool {w['P']} pages)",
            "input_copies": reps}
     res["fused"] = row(graph_time_ms([fused(d) for d in ds], iters, dev), nb["fused"])
-    if cfg in (2, 3):
+    if cfg in (2, 3, 5):
         res["select_only"] = row(graph_time_ms([select(d) for d in ds], iters, dev), vb["select"])
+        res["select_only_lossy"] = row(graph_time_ms([select_lossy(d) for d in ds], iters, dev),
+                                       vb["select"])
+    if cfg in (2, 3):
         for d in ds:
             select(d)()
         res["decode_only"] = row(graph_time_ms([decode(d) for d in ds], iters, dev), vb["decode"])
@@ -744,6 +783,9 @@ def main():
                     help="workload of the hot-path table (the headline line is config 2)")
     ap.add_argument("--plan", action="store_true",
                     help="add the vt_plan_requests launch to the step")
+    ap.add_argument("--step-mode", choices=["one-launch", "two-call"], default="one-launch",
+                    help="the step as one vt_sparse_decode_step launch, or vt_build_centroids "
+                         "beside vt_sparse_decode_fused on two streams")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per-workload rows (configs 1-5) of the default run")
