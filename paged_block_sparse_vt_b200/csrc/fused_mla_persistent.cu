@@ -37,7 +37,8 @@ constexpr int kMpRow = kMpD + 8;   // smem row stride of Q and K tiles (elements
 constexpr int kMlaChunk = 224;     // candidate pages per scan item (28 per warp)
 constexpr int kMpScanRows = 2;     // centroid rows per ring slot
 constexpr int kMpScanSlots = 5;    // ring slots per warp (4 landing while one is used)
-constexpr int kMpPiece = 8;        // most selected pages per attention item (one warp each)
+constexpr int kMpPiece = 32;       // most selected pages per attention item
+constexpr int kMpRound = 4;        // pages of a piece staged and computed together (64 tokens)
 constexpr int kMpMaxB = 2048;      // requests the persistent path takes
 
 // ---- sizes derived from the call ----------------------------------------------------------
@@ -110,7 +111,7 @@ static MpWsLayout mp_ws_layout(const DecodeParams& p, int G, int64_t unit_cap) {
 
 struct MpSmem {
   int prefix, keys, pids, qm, sel, phys, ml, misc, region;  // region: one phase at a time
-  int ring, q, kt, pm, pmax, psum;                          // region offsets
+  int ring, q, kt, pm, pmax, psum, fac;                     // region offsets
   int total;
 };
 
@@ -134,15 +135,16 @@ __host__ __device__ inline MpSmem mp_smem_layout(int G, int B, const MpGeom& g) 
   const int merge_small = 3 * 2 * kMpThreads * 4 + SmallTopk<kMpThreads>::BYTES;
   const int merge_big = align16(g.cmax * 4) + align16(g.cmax * 2) + align16((kTopkBins + 64) * 4);
   const int merge = merge_small > merge_big ? merge_small : merge_big;
-  // attention: the piece's K tiles (first: the merge scratch above is dead once they load),
-  // Q (prefetched while the merge runs), P, per-page maxima and sums
-  const int T = kMpPiece * kPage;
+  // attention: two buffers of a round's K tiles (first: the merge scratch above is dead once
+  // they load), Q (prefetched while the merge runs), P, per-page maxima and sums, rescales
+  const int RT = kMpRound * kPage;
   int a = 0;
-  s.kt = a; a += align16(T * kMpRow * 2);
+  s.kt = a; a += align16(2 * RT * kMpRow * 2);
   s.q = a;  a += align16(G * kMpRow * 2);
-  s.pm = a; a += align16(G * (T + 8) * 2);
-  s.pmax = a; a += align16(kMpPiece * G * 4);
-  s.psum = a; a += align16(kMpPiece * G * 4);
+  s.pm = a; a += align16(G * (RT + 8) * 2);
+  s.pmax = a; a += align16(kMpRound * G * 4);
+  s.psum = a; a += align16(kMpRound * G * 4);
+  s.fac = a; a += align16(G * 4);
   int r = scan;
   if (merge > r) r = merge;
   if (a > r) r = a;
@@ -180,11 +182,12 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
   constexpr int DV = kMpDv;
   constexpr int CH4 = D / 4;  // float4 per centroid row
   constexpr int RB = D * 4;   // bytes of a centroid row
-  constexpr int T = kMpPiece * kPage;
-  constexpr int PST = T + 8;
+  constexpr int RT = kMpRound * kPage;  // tokens of a round
+  constexpr int PST = RT + 8;
   static_assert(G == 16 || G == 32, "MLA path covers 16 or 32 query heads");
   static_assert(kMlaChunk <= 32 * kMpWarps, "one page id per lane: at most 32 rows per warp");
-  static_assert(kMpPiece >= 2, "the page-max table [kMpPiece][G] holds the merge's [G][2]");
+  static_assert(kMpRound >= 2, "the page-max table [kMpRound][G] holds the merge's [G][2]");
+  static_assert(kMpRound * 2 <= kMpWarps, "S^T: a warp per page of a round (two when G = 32)");
   static_assert(SmallTopk<NT>::BYTES <= kMpScanSlots * kMpScanRows * RB,
                 "the chunk top-k scratch fits in warp 0's ring");
 
@@ -259,6 +262,29 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
   const int total_items = scan_items + p.B * A;
   auto block_start = [&](int b) { return s_prefix[b] + A * max(0, b - lag); };
 
+  // item t: (scan, request, chunk) or (attention, request, piece)
+  auto decode = [&](int t, bool& is_scan, int& ib, int& ic) {
+    is_scan = false;
+    if (t >= block_start(p.B)) {
+      const int r = t - block_start(p.B);
+      ib = (p.B - lag) + r / A;
+      ic = r % A;
+    } else {
+      int lo = 0, hi = p.B - 1;  // the block holding t
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (block_start(mid) <= t) lo = mid; else hi = mid - 1;
+      }
+      const int r = t - block_start(lo), nc = s_prefix[lo + 1] - s_prefix[lo];
+      is_scan = r < nc;
+      ib = is_scan ? lo : lo - lag;
+      ic = is_scan ? r : r - nc;
+    }
+  };
+  // A scan item whose successor is a scan item loads the successor's page ids while its own
+  // top-k runs (pre_t, pre_pid), and consecutive chunks of one request keep its query mean in
+  // shared memory (qm_b): a chunk then starts streaming one round trip after it is taken.
+  int pre_t = -1, pre_pid = -1, qm_b = -1;
   int32_t* pending = nullptr;  // thread 0: a counter to bump after the item's closing barrier
   for (;;) {
     const int t = s_misc[0];
@@ -286,24 +312,9 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
       continue;
     }
 
-    // decode the item: (scan, request, chunk) or (attention, request, piece)
-    bool is_scan = false;
+    bool is_scan;
     int ib, ic;
-    if (t >= block_start(p.B)) {
-      const int r = t - block_start(p.B);
-      ib = (p.B - lag) + r / A;
-      ic = r % A;
-    } else {
-      int lo = 0, hi = p.B - 1;  // the block holding t
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (block_start(mid) <= t) lo = mid; else hi = mid - 1;
-      }
-      const int r = t - block_start(lo), nc = s_prefix[lo + 1] - s_prefix[lo];
-      is_scan = r < nc;
-      ib = is_scan ? lo : lo - lag;
-      ic = is_scan ? r : r - nc;
-    }
+    decode(t, is_scan, ib, ic);
     if (is_scan) {
       // ---------------------------------------------------------------- scan item
       const int b = ib, c = ic;
@@ -316,7 +327,7 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
       const int myrows = (cnt - warp + NW - 1) / NW;
       int pid = -1;
       if (lane < myrows) {
-        pid = ptrow[p.bos + c0 + warp + NW * lane];
+        pid = pre_t == t ? pre_pid : ptrow[p.bos + c0 + warp + NW * lane];
         if (pid < 0 || pid >= p.num_pages) {
           flag(p.status, VT_DEV_BAD_PAGE);
           pid = -1;
@@ -326,7 +337,8 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
       // fp32 mean of the request's G query heads: three groups of 72 threads each load every
       // third row (one round of independent 16-byte loads), then sum through shared memory
       const __nv_bfloat16* qb = p.q + (int64_t)b * p.Hq * D;
-      {
+      if (qm_b != b) {  // (uniform: every thread has seen the same items)
+        qm_b = b;
         constexpr int NC8 = D / 8;  // 16-byte chunks per query row
         float* s_part = reinterpret_cast<float*>(region);  // [3][D], in warp 0..2's rings, before use
         const int grp = tid / NC8, c8 = tid - grp * NC8;
@@ -417,7 +429,10 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
         __syncwarp();  // every lane is done with the slot before it is refilled
       }
       cp_async_wait<0>();
-      if (tid == 0) next = claim();
+      if (tid == 0) {
+        next = claim();
+        s_misc[2] = next;
+      }
       if (lane == 0) {
         s_misc[16 + warp] = (int)klo;
         s_misc[16 + NW + warp] = (int)khi;
@@ -427,6 +442,22 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
         for (int i = lane; i < SmallTopk<NT>::HIST / 4; i += 32)
           reinterpret_cast<int4*>(tk)[i] = make_int4(0, 0, 0, 0);
       __syncthreads();  // every score of the chunk is in s_keys; the rings are free
+      {  // a scan item next: its page ids are loaded now and land while this chunk's top-k runs
+        const int t2 = s_misc[2];
+        pre_t = -1;
+        bool sc2 = false;
+        int b2 = 0, c2 = 0;
+        if (t2 >= 0 && t2 < total_items) decode(t2, sc2, b2, c2);
+        if (sc2) {
+          const int n2 = (p.seq_lens[b2] + kPage - 1) / kPage;
+          const int c02 = c2 * kMlaChunk, cnt2 = min(kMlaChunk, n2 - p.bos - p.eos - c02);
+          const int myrows2 = (cnt2 - warp + NW - 1) / NW;
+          pre_pid = lane < myrows2
+                        ? p.page_table[(int64_t)b2 * p.pt_stride + p.bos + c02 + warp + NW * lane]
+                        : -1;
+          pre_t = t2;
+        }
+      }
       klo = 0xffffffffu;
       khi = 0u;
 #pragma unroll
@@ -589,126 +620,43 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
           if (tid < np) s_phys[tid] = phys_of(s_sel[tid]);
           __syncthreads();
         }
-        // ---- stage the piece's K tiles (zero rows past the valid tokens), and Q if not yet
-        __nv_bfloat16* s_kt = reinterpret_cast<__nv_bfloat16*>(region + Ls.kt);
-        __nv_bfloat16* s_pm = reinterpret_cast<__nv_bfloat16*>(region + Ls.pm);  // [G][T+8]
-        float* s_pmax = reinterpret_cast<float*>(region + Ls.pmax);             // [piece page][G]
-        float* s_psum = reinterpret_cast<float*>(region + Ls.psum);             // [piece page][G]
+        // ---- the piece's pages in rounds of kMpRound: K tiles (zero rows past the valid
+        // tokens) double-buffered, so that round r + 1 lands while round r computes; an online
+        // softmax carries each head's running maximum and sum from round to round
+        __nv_bfloat16* s_kt = reinterpret_cast<__nv_bfloat16*>(region + Ls.kt);  // [2][RT][kMpRow]
+        __nv_bfloat16* s_pm = reinterpret_cast<__nv_bfloat16*>(region + Ls.pm);  // [G][RT+8]
+        float* s_pmax = reinterpret_cast<float*>(region + Ls.pmax);             // [round page][G]
+        float* s_psum = reinterpret_cast<float*>(region + Ls.psum);             // [round page][G]
+        float* s_fac = reinterpret_cast<float*>(region + Ls.fac);               // [G]
+        float* s_run = s_ml;                                                     // [G][2]
         const int last_valid = L - kPage * (n - 1);
         if (!q_early) stage_q();
-        // warp w loads page w of the piece itself, so that its S^T can start as soon as its
-        // own tile has landed (every thread commits the group, empty or not)
-        if (warp < np) {
-          const int pg = s_phys[warp];
-          const bool lastp = s_sel[warp] == n - 1;
-          for (int i = lane; i < kPage * (D / 8); i += 32) {
-            const int tt = i / (D / 8), c8 = i - tt * (D / 8);
-            const bool ok_row = pg >= 0 && (!lastp || tt < last_valid);
-            const __nv_bfloat16* src =
-                ok_row ? p.k_pool + (int64_t)pg * p.sk_p + (int64_t)tt * p.sk_t + c8 * 8 : p.k_pool;
-            cp_async16(smem_u32(s_kt + (warp * 16 + tt) * kMpRow + c8 * 8), src, ok_row ? 16 : 0);
-          }
-        }
-        cp_async_commit();
-        cp_async_wait<1>();  // this thread's share of Q has landed
-        __syncthreads();     // all of Q has
-        cp_async_wait<0>();  // and this warp's page
-        __syncwarp();
-        // ---- S^T = K Q^T: warp w owns page w (16 tokens) x all G heads, kept in registers:
-        // this lane holds tokens r0 = lane/4 and r0 + 8, heads nt*8 + 2 (lane%4) + {0, 1}
-        float acc[G / 8][4];
-#pragma unroll
-        for (int nt = 0; nt < G / 8; ++nt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
-        if (warp < np) {
-          const uint32_t a_base = smem_u32(s_kt + (warp * 16 + (lane & 15)) * kMpRow + (lane >> 4) * 8);
-          const uint32_t b_base =
-              smem_u32(s_q + ((lane & 7) + ((lane >> 4) << 3)) * kMpRow + ((lane >> 3) & 1) * 8);
-#pragma unroll 4
-          for (int ks = 0; ks < D / 16; ++ks) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(a_base + ks * 32, a0, a1, a2, a3);
-#pragma unroll
-            for (int n2 = 0; n2 < G / 16; ++n2) {
-              uint32_t b0, b1, b2, b3;
-              ldsm_x4(b_base + n2 * 16 * kMpRow * 2 + ks * 32, b0, b1, b2, b3);
-              mma_16816(acc[2 * n2], a0, a1, a2, a3, b0, b1);
-              mma_16816(acc[2 * n2 + 1], a0, a1, a2, a3, b2, b3);
+        const int nr = (np + kMpRound - 1) / kMpRound;
+        auto row_ok = [&](int j, int tt) {  // token tt of the piece's j-th page is attended
+          return j < np && s_phys[j] >= 0 && (s_sel[j] != n - 1 || tt < last_valid);
+        };
+        auto stage_round = [&](int r) {  // every thread commits one group per call
+          if (r < nr) {
+            __nv_bfloat16* dst = s_kt + (r & 1) * RT * kMpRow;
+            constexpr int C8 = D / 8;  // 16-byte chunks per K row
+            for (int i = tid; i < RT * C8; i += NT) {
+              const int row = i / C8, c8 = i - row * C8;
+              const int j = r * kMpRound + row / kPage, tt = row % kPage;
+              const bool ok_row = row_ok(j, tt);
+              const __nv_bfloat16* src =
+                  ok_row ? p.k_pool + (int64_t)s_phys[j] * p.sk_p + (int64_t)tt * p.sk_t + c8 * 8
+                         : p.k_pool;
+              cp_async16(smem_u32(dst + row * kMpRow + c8 * 8), src, ok_row ? 16 : 0);
             }
           }
-        }
-        // ---- softmax over the piece's tokens, per head: page maxima, then probabilities
-        // against the piece's maximum (rounded once to bf16, as the P V MMA reads them)
-        const int r0 = lane >> 2;
-        bool v0 = false, v1 = false;
-        if (warp < np) {
-          const bool live = s_phys[warp] >= 0, lastp = s_sel[warp] == n - 1;
-          v0 = live && (!lastp || r0 < last_valid);
-          v1 = live && (!lastp || r0 + 8 < last_valid);
-        }
-#pragma unroll
-        for (int nt = 0; nt < G / 8; ++nt) {
-          acc[nt][0] = v0 ? acc[nt][0] * p.qscale : -INFINITY;
-          acc[nt][1] = v0 ? acc[nt][1] * p.qscale : -INFINITY;
-          acc[nt][2] = v1 ? acc[nt][2] * p.qscale : -INFINITY;
-          acc[nt][3] = v1 ? acc[nt][3] * p.qscale : -INFINITY;
-          float m0 = fmaxf(acc[nt][0], acc[nt][2]), m1 = fmaxf(acc[nt][1], acc[nt][3]);
-#pragma unroll
-          for (int o = 4; o <= 16; o <<= 1) {
-            m0 = fmaxf(m0, __shfl_xor_sync(kFull, m0, o));
-            m1 = fmaxf(m1, __shfl_xor_sync(kFull, m1, o));
-          }
-          if (warp < np && lane < 4) {
-            s_pmax[warp * G + nt * 8 + 2 * lane] = m0;
-            s_pmax[warp * G + nt * 8 + 2 * lane + 1] = m1;
-          }
-        }
-        __syncthreads();
-        if (warp < np) {
-#pragma unroll
-          for (int nt = 0; nt < G / 8; ++nt) {
-            const int c = nt * 8 + 2 * (lane & 3);
-            float M0 = -INFINITY, M1 = -INFINITY;
-            for (int q = 0; q < np; ++q) {
-              M0 = fmaxf(M0, s_pmax[q * G + c]);
-              M1 = fmaxf(M1, s_pmax[q * G + c + 1]);
-            }
-            const __nv_bfloat16 p00 = __float2bfloat16(acc[nt][0] == -INFINITY ? 0.0f : exp2f(acc[nt][0] - M0));
-            const __nv_bfloat16 p01 = __float2bfloat16(acc[nt][1] == -INFINITY ? 0.0f : exp2f(acc[nt][1] - M1));
-            const __nv_bfloat16 p10 = __float2bfloat16(acc[nt][2] == -INFINITY ? 0.0f : exp2f(acc[nt][2] - M0));
-            const __nv_bfloat16 p11 = __float2bfloat16(acc[nt][3] == -INFINITY ? 0.0f : exp2f(acc[nt][3] - M1));
-            const int tk = warp * 16 + r0;
-            s_pm[c * PST + tk] = p00;
-            s_pm[(c + 1) * PST + tk] = p01;
-            s_pm[c * PST + tk + 8] = p10;
-            s_pm[(c + 1) * PST + tk + 8] = p11;
-            // the sums use the rounded weights, as the MMA does
-            float l0 = __bfloat162float(p00) + __bfloat162float(p10);
-            float l1 = __bfloat162float(p01) + __bfloat162float(p11);
-#pragma unroll
-            for (int o = 4; o <= 16; o <<= 1) {
-              l0 += __shfl_xor_sync(kFull, l0, o);
-              l1 += __shfl_xor_sync(kFull, l1, o);
-            }
-            if (lane < 4) {
-              s_psum[warp * G + c] = l0;
-              s_psum[warp * G + c + 1] = l1;
-            }
-          }
-        }
-        __syncthreads();
+          cp_async_commit();
+        };
+        stage_round(0);
+        stage_round(1);
         for (int g = tid; g < G; g += NT) {
-          float M = -INFINITY, Ls = 0.0f;
-          for (int q = 0; q < np; ++q) {
-            M = fmaxf(M, s_pmax[q * G + g]);
-            Ls += s_psum[q * G + g];
-          }
-          s_ml[2 * g] = M;
-          s_ml[2 * g + 1] = Ls;
+          s_run[2 * g] = -INFINITY;
+          s_run[2 * g + 1] = 0.0f;
         }
-        __syncthreads();
-        // ---- O = P V: warp w owns output dims [64 w, 64 w + 64) for all G heads
         float oacc[G / 16][8][4];
 #pragma unroll
         for (int mt = 0; mt < G / 16; ++mt)
@@ -716,27 +664,146 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
           for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) oacc[mt][nt][i] = 0.0f;
-        {
-          const uint32_t pa_base = smem_u32(s_pm + (lane & 15) * PST + (lane >> 4) * 8);
-          const uint32_t vb_base = smem_u32(s_kt + ((lane & 7) + ((lane >> 3) & 1) * 8) * kMpRow +
-                                            warp * 64 + (lane >> 4) * 8);
-          for (int ks = 0; ks < np; ++ks) {  // 16 tokens per step
-            uint32_t ar[G / 16][4];
+        // S^T: warp w takes page w % kMpRound of the round and 16 of the heads (the second
+        // half of them on warps kMpRound.. when G = 32); its lane holds tokens r0 = lane/4
+        // and r0 + 8, heads hb + nt*8 + 2 (lane%4) + {0, 1}
+        constexpr int SPLIT = G / 16;  // warps per page in S^T
+        const int spage = warp % kMpRound, hb = (warp / kMpRound) * 16;
+        const bool s_warp = warp < kMpRound * SPLIT;
+        const int r0 = lane >> 2;
+        for (int r = 0; r < nr; ++r) {
+          cp_async_wait<1>();  // this thread's share of round r (and of Q) has landed
+          __syncthreads();     // everyone's has; the running statistics are initialised
+          const __nv_bfloat16* kt = s_kt + (r & 1) * RT * kMpRow;
+          const int j = r * kMpRound + spage;  // the piece's page this warp scores
+          float acc[2][4];
 #pragma unroll
-            for (int mt = 0; mt < G / 16; ++mt)
-              ldsm_x4(pa_base + (mt * 16 * PST + ks * 16) * 2, ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3]);
+          for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int n2 = 0; n2 < 4; ++n2) {
-              uint32_t b0, b1, b2, b3;
-              ldsm_x4_t(vb_base + (ks * 16 * kMpRow + n2 * 16) * 2, b0, b1, b2, b3);
+            for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+          if (s_warp && j < np) {
+            const uint32_t a_base =
+                smem_u32(kt + (spage * 16 + (lane & 15)) * kMpRow + (lane >> 4) * 8);
+            const uint32_t b_base = smem_u32(
+                s_q + (hb + (lane & 7) + ((lane >> 4) << 3)) * kMpRow + ((lane >> 3) & 1) * 8);
+#pragma unroll 4
+            for (int ks = 0; ks < D / 16; ++ks) {
+              uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+              ldsm_x4(a_base + ks * 32, a0, a1, a2, a3);
+              ldsm_x4(b_base + ks * 32, b0, b1, b2, b3);
+              mma_16816(acc[0], a0, a1, a2, a3, b0, b1);
+              mma_16816(acc[1], a0, a1, a2, a3, b2, b3);
+            }
+          }
+          // page maxima per head (base 2, masked tokens -inf)
+          const bool v0 = s_warp && row_ok(j, r0), v1 = s_warp && row_ok(j, r0 + 8);
 #pragma unroll
-              for (int mt = 0; mt < G / 16; ++mt) {
-                mma_16816(oacc[mt][2 * n2], ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3], b0, b1);
-                mma_16816(oacc[mt][2 * n2 + 1], ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3], b2, b3);
+          for (int nt = 0; nt < 2; ++nt) {
+            acc[nt][0] = v0 ? acc[nt][0] * p.qscale : -INFINITY;
+            acc[nt][1] = v0 ? acc[nt][1] * p.qscale : -INFINITY;
+            acc[nt][2] = v1 ? acc[nt][2] * p.qscale : -INFINITY;
+            acc[nt][3] = v1 ? acc[nt][3] * p.qscale : -INFINITY;
+            float m0 = fmaxf(acc[nt][0], acc[nt][2]), m1 = fmaxf(acc[nt][1], acc[nt][3]);
+#pragma unroll
+            for (int o = 4; o <= 16; o <<= 1) {
+              m0 = fmaxf(m0, __shfl_xor_sync(kFull, m0, o));
+              m1 = fmaxf(m1, __shfl_xor_sync(kFull, m1, o));
+            }
+            if (s_warp && lane < 4) {
+              s_pmax[spage * G + hb + nt * 8 + 2 * lane] = m0;
+              s_pmax[spage * G + hb + nt * 8 + 2 * lane + 1] = m1;
+            }
+          }
+          __syncthreads();
+          // probabilities against the new running maximum (rounded once to bf16, as the P V
+          // MMA reads them) and their sums per page and head
+          if (s_warp) {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              const int c = hb + nt * 8 + 2 * (lane & 3);
+              float M0 = s_run[2 * c], M1 = s_run[2 * (c + 1)];
+#pragma unroll
+              for (int q = 0; q < kMpRound; ++q) {
+                M0 = fmaxf(M0, s_pmax[q * G + c]);
+                M1 = fmaxf(M1, s_pmax[q * G + c + 1]);
+              }
+              const __nv_bfloat16 p00 = __float2bfloat16(acc[nt][0] == -INFINITY ? 0.0f : exp2f(acc[nt][0] - M0));
+              const __nv_bfloat16 p01 = __float2bfloat16(acc[nt][1] == -INFINITY ? 0.0f : exp2f(acc[nt][1] - M1));
+              const __nv_bfloat16 p10 = __float2bfloat16(acc[nt][2] == -INFINITY ? 0.0f : exp2f(acc[nt][2] - M0));
+              const __nv_bfloat16 p11 = __float2bfloat16(acc[nt][3] == -INFINITY ? 0.0f : exp2f(acc[nt][3] - M1));
+              const int tk = spage * 16 + r0;
+              s_pm[c * PST + tk] = p00;
+              s_pm[(c + 1) * PST + tk] = p01;
+              s_pm[c * PST + tk + 8] = p10;
+              s_pm[(c + 1) * PST + tk + 8] = p11;
+              // the sums use the rounded weights, as the MMA does
+              float l0 = __bfloat162float(p00) + __bfloat162float(p10);
+              float l1 = __bfloat162float(p01) + __bfloat162float(p11);
+#pragma unroll
+              for (int o = 4; o <= 16; o <<= 1) {
+                l0 += __shfl_xor_sync(kFull, l0, o);
+                l1 += __shfl_xor_sync(kFull, l1, o);
+              }
+              if (lane < 4) {
+                s_psum[spage * G + c] = l0;
+                s_psum[spage * G + c + 1] = l1;
               }
             }
           }
+          __syncthreads();
+          // the running statistics move to the new maximum; O is rescaled by s_fac below
+          for (int g = tid; g < G; g += NT) {
+            const float Mo = s_run[2 * g];
+            float Mn = Mo, Ls = 0.0f;
+            for (int q = 0; q < kMpRound; ++q) {
+              Mn = fmaxf(Mn, s_pmax[q * G + g]);
+              Ls += s_psum[q * G + g];
+            }
+            const float f = (Mo == -INFINITY) ? 0.0f : exp2f(Mo - Mn);
+            s_fac[g] = f;
+            s_run[2 * g] = Mn;
+            s_run[2 * g + 1] = fmaf(s_run[2 * g + 1], f, Ls);
+          }
+          __syncthreads();
+          // O += P V over the round's tokens: warp w owns output dims [64 w, 64 w + 64) for
+          // all G heads; V is the first 512 dims of the staged K rows
+#pragma unroll
+          for (int mt = 0; mt < G / 16; ++mt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const float f = s_fac[mt * 16 + (lane >> 2) + 8 * hh];
+#pragma unroll
+              for (int nt = 0; nt < 8; ++nt) {
+                oacc[mt][nt][2 * hh] *= f;
+                oacc[mt][nt][2 * hh + 1] *= f;
+              }
+            }
+          {
+            const int pr = min(kMpRound, np - r * kMpRound);  // pages of this round
+            const uint32_t pa_base = smem_u32(s_pm + (lane & 15) * PST + (lane >> 4) * 8);
+            const uint32_t vb_base = smem_u32(kt + ((lane & 7) + ((lane >> 3) & 1) * 8) * kMpRow +
+                                              warp * 64 + (lane >> 4) * 8);
+            for (int ks = 0; ks < pr; ++ks) {  // 16 tokens per step
+              uint32_t ar[G / 16][4];
+#pragma unroll
+              for (int mt = 0; mt < G / 16; ++mt)
+                ldsm_x4(pa_base + (mt * 16 * PST + ks * 16) * 2, ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3]);
+#pragma unroll
+              for (int n2 = 0; n2 < 4; ++n2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(vb_base + (ks * 16 * kMpRow + n2 * 16) * 2, b0, b1, b2, b3);
+#pragma unroll
+                for (int mt = 0; mt < G / 16; ++mt) {
+                  mma_16816(oacc[mt][2 * n2], ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3], b0, b1);
+                  mma_16816(oacc[mt][2 * n2 + 1], ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3], b2, b3);
+                }
+              }
+            }
+          }
+          __syncthreads();  // every warp is done with this buffer and with P
+          stage_round(r + 2);
         }
+        cp_async_wait<0>();
         // ---- finish: this lane holds heads g = 16 mt + lane/4 (+8), dims 64 warp + 8 nt + 2 (lane%4) (+1)
         auto write_out = [&](float (&o)[G / 16][8][4], auto&& ml_of) {
 #pragma unroll

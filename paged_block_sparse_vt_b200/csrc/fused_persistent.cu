@@ -624,7 +624,7 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
               klo = min(klo, (uint32_t)s_misc[16 + k]);
               khi = max(khi, (uint32_t)s_misc[16 + NW + k]);
             }
-            small_topk<NT>(keys, C, topk, klo, khi, tk, [&](int j, int pos) {
+            auto put = [&](int j, int pos) {
               const int q = bos + pos - j0;
               if (q >= 0 && q < np) {
                 s_sel[q] = lps[j];
@@ -636,7 +636,8 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
                 s_phys[q] = pg;
               }
               if (write_sel) selrow[bos + pos] = lps[j];
-            });
+            };
+            small_topk<NT>(keys, C, topk, klo, khi, tk, put);
             have_phys = true;
           } else {
             if (rlp >= 0) s_sel[tid] = rlp;  // page ids of the whole piece are looked up below
