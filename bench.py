@@ -22,6 +22,7 @@ finds its data in L2.  Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -552,6 +553,10 @@ def run_ours(args, world, rank, local):
             per_config[str(cfg)] = measure_config(vt, cfg, dev, peak)
             log(f"config {cfg}: {time.perf_counter() - t0:.1f} s, fused "
                 f"{per_config[str(cfg)]['fused']['us']} us")
+        t0 = time.perf_counter()
+        per_config["serving_pass"] = measure_serving_pass(vt, dev, peak)
+        log(f"serving pass: {time.perf_counter() - t0:.1f} s, "
+            f"{per_config['serving_pass']['pass_us']} us")
         per_config["clocks"] = pc_clocks.stop()
         per_config["timing"] = ("per row: 10 calls captured as one CUDA graph, one untimed "
                                 "replay, one replay between CUDA events; us = per call")
@@ -721,6 +726,99 @@ def measure_config(vt, cfg: int, dev, peak: float, iters: int = 10) -> dict:
     if any(int(d["status"].item()) for d in ds):
         raise SystemExit(f"config {cfg}: device status set: an input was rejected by the kernels")
     del ds
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_serving_pass(vt, dev, peak: float, L: int = 28, copies: int = 3) -> dict:
+    """A serving-shaped decode pass over the Qwen3-0.6B-like batch: L layers, each one
+    vt_sparse_decode_step launch (the build of the pages filled at this step, then select +
+    attend), layer 0 dense (every page attended: the README runs its sparse attention with
+    vortex_layers_skip = [0]), captured as one CUDA graph as a serving engine captures its
+    decode step.  Layer l has its own query and reads K/V pool copy l % copies (each with its
+    own centroid cache): the copies hold 3 x 2.6 GB, so no layer finds its data in L2."""
+    c = config(2)
+    w = make_workload(c, seed=1002)
+    dense_topk = int(w["page_table"].shape[1])  # >= every request's candidates
+    pools = []
+    for r in range(copies):
+        d = {k: w[k].to(dev) for k in ("k_pool", "v_pool", "page_table", "seq_lens",
+                                       "prebuilt_pages", "fill_pages")}
+        d["cent"] = torch.zeros((w["P"], c.Hkv, c.D), dtype=torch.float32, device=dev)
+        vt.vt_build_centroids(d["k_pool"], d["prebuilt_pages"], d["cent"])
+        pools.append(d)
+    g = torch.Generator().manual_seed(77)
+    layers = []
+    for l in range(L):
+        d = dict(pools[l % copies])
+        d["q"] = torch.randn((c.B, c.Hq, c.D), generator=g).to(torch.bfloat16).to(dev)
+        d["topk"] = dense_topk if l == 0 else c.topk
+        d["out"] = torch.empty((c.B, c.Hq, c.Dv), dtype=torch.bfloat16, device=dev)
+        d["lse"] = torch.empty((c.B, c.Hq), dtype=torch.float32, device=dev)
+        d["status"] = torch.zeros((1,), dtype=torch.int32, device=dev)
+        d["ws"] = vt.fused_workspace(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                     d["seq_lens"], d["cent"], d["topk"], c.bos, c.eos)
+        layers.append(d)
+    torch.cuda.synchronize(dev)
+
+    def layer_call(d):
+        return lambda: vt.vt_sparse_decode_step(
+            d["q"], d["k_pool"], d["v_pool"], d["page_table"], d["seq_lens"], d["cent"],
+            d["topk"], c.bos, c.eos, c.sm_scale, d["fill_pages"], out=d["out"], lse=d["lse"],
+            status=d["status"], workspace=d["ws"])
+
+    calls = [layer_call(d) for d in layers]
+    pass_us = graph_time_ms([lambda: [f() for f in calls]], 3, dev) * 1e3
+    dense_us = graph_time_ms([calls[0]], 6, dev) * 1e3
+    sparse_us = graph_time_ms(calls[1:], 3 * (L - 1), dev) * 1e3
+    if any(int(d["status"].item()) for d in layers):
+        raise SystemExit("serving pass: device status set")
+    nb = algorithmic_bytes(c, w["seq_lens"])
+    dense_cfg = dataclasses.replace(c, topk=dense_topk)
+    nbd = algorithmic_bytes(dense_cfg, w["seq_lens"])
+    # end to end: the step's host inputs (page tables, lengths, filled pages) in, the pass, the
+    # last layer's output back, per pass (the queries of later layers come from the model on
+    # the device)
+    host = [w[k].pin_memory() for k in ("page_table", "seq_lens", "fill_pages")]
+    out_h = torch.empty_like(layers[-1]["out"], device="cpu").pin_memory()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for f in calls:
+            f()
+    gr.replay()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    h2d = sum(t.numel() * t.element_size() for t in host)
+
+    def e2e_pass():
+        for d in pools:
+            for t, k in zip(host, ("page_table", "seq_lens", "fill_pages")):
+                d[k].copy_(t, non_blocking=True)
+        gr.replay()
+        out_h.copy_(layers[-1]["out"], non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(3):
+        e2e_pass()
+    t0 = time.perf_counter()
+    reps = 10
+    for _ in range(reps):
+        e2e_pass()
+    e2e_us = (time.perf_counter() - t0) / reps * 1e6
+    res = {
+        "workload": f"{L}-layer decode pass of the {c.name} batch (layer 0 dense, layers 1.."
+                    f"{L - 1} top-{c.topk}+{c.bos}+{c.eos}), one vt_sparse_decode_step launch "
+                    f"per layer, captured as one CUDA graph",
+        "layers": L, "pass_us": round(pass_us, 1),
+        "sparse_layer_us": round(sparse_us, 2), "dense_layer_us": round(dense_us, 2),
+        "sparse_layer_frac": round(nb["total"] / (sparse_us / 1e6) / 1e9 / peak, 4),
+        "dense_layer_frac": round(nbd["total"] / (dense_us / 1e6) / 1e9 / peak, 4),
+        "tokens_per_s": c.B / (pass_us / 1e6),
+        "e2e": {"pass_us": round(e2e_us, 1), "tokens_per_s": c.B / (e2e_us / 1e6),
+                "h2d_bytes_per_pass": h2d * len(pools),
+                "d2h_bytes_per_pass": out_h.numel() * out_h.element_size()},
+    }
+    del gr, layers, pools
     torch.cuda.empty_cache()
     return res
 

@@ -10,18 +10,22 @@
 // q_lat . c_lat + q_rope . c_rope is one dot product over the 576-dim row (the page mean is
 // linear in each part).
 //
-// One CTA of 8 warps per SM (the attention stages Q and eight K tiles: ~210 KB).  Items:
+// One CTA of 8 warps per SM (the attention stages Q and two buffers of four K tiles: ~200 KB).
+// Items:
+//   build items  -- (vt_sparse_decode_step only) the centroid of one page filled at this step;
 //   scan items   -- (request, chunk of kMlaChunk candidate pages): each warp streams its rows
 //                   of fp32 centroids (2304 B each) through a cp.async ring and dots them with
 //                   the fp32 mean of the request's query heads; the CTA keeps the chunk's exact
 //                   top-k (key, offset, page id) and counts the chunk done;
-//   attention    -- (request, piece of <= 8 selected pages): waits until every chunk of the
-//   items           request is counted, merges the chunks' candidates with the same exact
-//                   top-k, stages Q and the piece's K tiles once in shared memory and runs
-//                   S^T = K Q^T (one warp per page), the softmax over the piece's tokens and
-//                   O = P V (each warp owns 64 of the 512 output dims) on the tensor cores;
-//                   with several pieces, the last one waits for the others' partials in the
-//                   workspace and merges them in registers.
+//   attention    -- (request, piece of <= kMpPiece selected pages): waits until every chunk of
+//   items           the request is counted, merges the chunks' candidates with the same exact
+//                   top-k, then takes the piece's pages in rounds of kMpRound: their K tiles
+//                   land in one buffer while the previous round computes from the other;
+//                   S^T = K Q^T (two warps per page, 16 heads each), the softmax against each
+//                   head's running maximum, and O = P V (each warp owns 64 of the 512 output
+//                   dims, rescaled when the maximum moves) on the tensor cores; with several
+//                   pieces, the last one waits for the others' partials in the workspace and
+//                   merges them in registers.
 // Queue, claims and counters work as in the GQA persistent kernel (fused_persistent.cu).
 #include "centroid_chunk.cuh"
 #include "decode_params.cuh"
@@ -34,7 +38,7 @@ constexpr int kMpWarps = kMpThreads / 32;
 constexpr int kMpD = 576;
 constexpr int kMpDv = 512;
 constexpr int kMpRow = kMpD + 8;   // smem row stride of Q and K tiles (elements): conflict-free ldmatrix
-constexpr int kMlaChunk = 224;     // candidate pages per scan item (28 per warp)
+constexpr int kMlaChunk = 256;     // candidate pages per scan item (32 per warp)
 constexpr int kMpScanRows = 2;     // centroid rows per ring slot
 constexpr int kMpScanSlots = 5;    // ring slots per warp (4 landing while one is used)
 constexpr int kMpPiece = 32;       // most selected pages per attention item
@@ -252,9 +256,10 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
   // of request b - lag, and the pieces of the last lag requests come at the end.  The
   // attention (tensor-core bound here) then overlaps the scans (HBM bound) of later requests,
   // and a request's chunks are about five rounds of CTAs ahead of its pieces (measured on the
-  // 64-request latent workload with 224-page chunks: 1 round 107.2 us, 2 rounds 95.6, 3 rounds
-  // 93.9, 5 rounds 93.1, 8 rounds 93.2, every scan first 93.4).  Every wait is still for items
-  // earlier in the queue.
+  // 64-request latent workload with eight-page pieces and 224-page chunks: 1 round 107.2 us,
+  // 2 rounds 95.6, 3 rounds 93.9, 5 rounds 93.1, 8 rounds 93.2, every scan first 93.4; with
+  // 17-page pieces and 256-page chunks 2 / 3 / 5 rounds gave 84.0 / 75.0 / 75.1 us).  Every
+  // wait is still for items earlier in the queue.
   const int scan_items = s_prefix[p.B];
   const int A = gm.A;
   const int avg = (scan_items + p.B - 1) / p.B;
@@ -323,7 +328,7 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
       const int m = n - p.bos - p.eos;
       const int c0 = c * kMlaChunk, cnt = min(kMlaChunk, m - c0);
       const int32_t* ptrow = p.page_table + (int64_t)b * p.pt_stride;
-      // warp w: rows w + NW i (i < 28) of the chunk; lane i < 28 holds the page id of row i
+      // warp w: rows w + NW i (i < 32) of the chunk; lane i holds the page id of row i
       const int myrows = (cnt - warp + NW - 1) / NW;
       int pid = -1;
       if (lane < myrows) {
