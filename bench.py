@@ -525,14 +525,14 @@ def run_ours(args, world, rank, local):
     in_ready = [torch.cuda.Event() for _ in reps]
     res_ready = torch.cuda.Event()
 
-    def h2d(i):
+    def copy_in(i):
         d = reps[i % args.replicas]
         with torch.cuda.stream(copy_stream):
             d["in_buf"].copy_(in_h, non_blocking=True)
             in_ready[i % args.replicas].record(copy_stream)
 
     def e2e_run(n):
-        h2d(0)
+        copy_in(0)
         for i in range(n):
             d = reps[i % args.replicas]
             stream.wait_event(in_ready[i % args.replicas])
@@ -540,7 +540,7 @@ def run_ours(args, world, rank, local):
                  after_fused=lambda d: out_h.copy_(d["out_buf"], non_blocking=True))
             res_ready.record(stream)
             if i + 1 < n:
-                h2d(i + 1)
+                copy_in(i + 1)
             res_ready.synchronize()  # the host has this step's result
 
     e2e_run(args.warmup)
@@ -695,6 +695,18 @@ def measure_config(vt, cfg: int, dev, peak: float, iters: int = 10) -> dict:
                                           sel=d["sel"], n_sel=d["n_sel"], status=d["status"],
                                           head_dim_v=c.Dv)
 
+    def select_ws(d):
+        return lambda: vt.vt_select_pages(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                          d["seq_lens"], d["cent"], c.topk, c.bos, c.eos,
+                                          sel=d["sel"], n_sel=d["n_sel"], status=d["status"],
+                                          head_dim_v=c.Dv, workspace=d["ws"])
+
+    def decode_ws(d):
+        return lambda: vt.vt_sparse_decode(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                           d["seq_lens"], d["sel"], d["n_sel"], c.sm_scale,
+                                           out=d["out"], lse=d["lse"], status=d["status"],
+                                           head_dim_v=c.Dv, workspace=d["ws_dec"])
+
     def select_lossy(d):
         return lambda: vt.vt_select_pages_approx(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
                                                  d["seq_lens"], d["cent"], c.topk, c.bos, c.eos,
@@ -719,6 +731,8 @@ def measure_config(vt, cfg: int, dev, peak: float, iters: int = 10) -> dict:
     res["fused"] = row(graph_time_ms([fused(d) for d in ds], iters, dev), nb["fused"])
     if cfg in (2, 3, 5):
         res["select_only"] = row(graph_time_ms([select(d) for d in ds], iters, dev), vb["select"])
+        res["select_only_workspace"] = row(graph_time_ms([select_ws(d) for d in ds], iters, dev),
+                                           vb["select"])
         res["select_only_lossy"] = row(graph_time_ms([select_lossy(d) for d in ds], iters, dev),
                                        vb["select"])
     if cfg in (2, 3):
@@ -728,6 +742,14 @@ def measure_config(vt, cfg: int, dev, peak: float, iters: int = 10) -> dict:
         res["select_then_decode"] = row(
             graph_time_ms([(lambda d=d: (select(d)(), decode(d)())) for d in ds], iters, dev),
             vb["select"] + vb["decode"])
+        for d in ds:
+            d["ws_dec"] = vt.decode_workspace(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                              d["seq_lens"], d["sel"], head_dim_v=c.Dv)
+        res["decode_only_workspace"] = row(graph_time_ms([decode_ws(d) for d in ds], iters, dev),
+                                           vb["decode"])
+        res["select_then_decode_workspace"] = row(
+            graph_time_ms([(lambda d=d: (select_ws(d)(), decode_ws(d)())) for d in ds], iters,
+                          dev), vb["select"] + vb["decode"])
     n_fill = int(w["fill_pages"].numel())
     if n_fill:
         d = ds[0]

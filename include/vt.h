@@ -142,6 +142,18 @@ vt_status vt_select_pages(const vt_paged_kv* kv, const vt_decode_args* a, int32_
                           int32_t* n_sel, void* stream);
 
 /*
+ * vt_select_pages with a workspace (vt_fused_workspace_size() bytes, 256-byte aligned, zeroed
+ * once, shared with the fused call under the same rules): for GQA heads and B <= 2048 the
+ * selection then runs on the fused call's persistent CTAs, scan items only, the unit's last
+ * counted chunk merging its candidates ("a workload planner for balanced GPU scheduling",
+ * rndamp.com article, "A dual-stage programmable abstraction").  Same results and errors as
+ * vt_select_pages; without a workspace, or for the MLA form, it is vt_select_pages.
+ */
+vt_status vt_select_pages_ws(const vt_paged_kv* kv, const vt_decode_args* a, int32_t* sel,
+                             int32_t* n_sel, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/*
  * The indexer's lossy mode ("stochastic radix top-k": a lossy, early-terminating top-k for
  * the indexing stage, rndamp.com article, "A dual-stage programmable abstraction"), as
  * vt_select_pages with the exact top-k replaced by one radix pass that stops there:
@@ -171,6 +183,16 @@ vt_status vt_select_pages_approx(const vt_paged_kv* kv, const vt_decode_args* a,
  */
 vt_status vt_sparse_decode(const vt_paged_kv* kv, const vt_decode_args* a, const int32_t* sel,
                            const int32_t* n_sel, void* out, float* lse, void* stream);
+
+/*
+ * vt_sparse_decode with a workspace (as for vt_select_pages_ws): for GQA heads and B <= 2048
+ * the attention then runs on the fused call's persistent CTAs, attention items only, reading
+ * the given selection.  Same results and errors as vt_sparse_decode; without a workspace, or
+ * for the MLA form, it is vt_sparse_decode.
+ */
+vt_status vt_sparse_decode_ws(const vt_paged_kv* kv, const vt_decode_args* a, const int32_t* sel,
+                              const int32_t* n_sel, void* out, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream);
 
 /*
  * The whole query side in one call: selection + attention ("kernel fusion",
@@ -219,8 +241,9 @@ vt_status vt_sparse_decode_step(const vt_paged_kv* kv, const vt_decode_args* a,
 /*
  * Bytes of workspace vt_sparse_decode_fused needs for these arguments (0 if
  * none); depends only on the shapes (B, Hq, Hkv, head dims, pt_stride, topk,
- * bos, eos), not on the data.  Returns 0 as well for arguments that
- * vt_sparse_decode_fused would reject.
+ * bos, eos), not on the data (args->centroids may be NULL).  Returns 0 as
+ * well for arguments that vt_sparse_decode_fused would reject otherwise.  It sizes the
+ * workspace of vt_select_pages_ws and vt_sparse_decode_ws too, for their own arguments.
  */
 size_t vt_fused_workspace_size(const vt_paged_kv* kv, const vt_decode_args* a);
 

@@ -16,6 +16,7 @@ from .binding import (  # noqa: F401
     VT_DEV_TIMEOUT,
     VtError,
     fused_workspace,
+    decode_workspace,
     load_library,
     prepare_build_centroids,
     prepare_sparse_decode_fused,

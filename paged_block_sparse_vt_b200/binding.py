@@ -51,6 +51,7 @@ class DecodeArgs(ctypes.Structure):
 
 
 EXPORTS = ("vt_build_centroids", "vt_select_pages", "vt_select_pages_approx",
+           "vt_select_pages_ws", "vt_sparse_decode_ws",
            "vt_sparse_decode", "vt_sparse_decode_fused", "vt_sparse_decode_step",
            "vt_fused_workspace_size", "vt_sparse_decode_fused_static", "vt_plan_requests",
            "vt_status_string",
@@ -78,6 +79,8 @@ def load_library(path: str = LIB_PATH):
                 "vt_build_centroids": [kv, P, I32, P, P, P],
                 "vt_select_pages": [kv, args, P, P, P],
                 "vt_select_pages_approx": [kv, args, ctypes.c_uint64, P, P, P],
+                "vt_select_pages_ws": [kv, args, P, P, P, ctypes.c_size_t, P],
+                "vt_sparse_decode_ws": [kv, args, P, P, P, P, P, ctypes.c_size_t, P],
                 "vt_sparse_decode": [kv, args, P, P, P, P, P],
                 "vt_sparse_decode_fused": [kv, args, P, P, P, P, P, ctypes.c_size_t, P],
                 "vt_sparse_decode_step": [kv, args, P, I32, P, P, P, P, P, P, ctypes.c_size_t, P],
@@ -182,8 +185,12 @@ def vt_build_centroids(k_pool: torch.Tensor, pages: torch.Tensor, centroids: tor
 
 
 def vt_select_pages(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos, eos,
-                    sel=None, n_sel=None, order=None, status=None, head_dim_v=None):
-    """Top-k page selection per (request, KV head).  Returns (sel [B,Hkv,kmax], n_sel [B,Hkv])."""
+                    sel=None, n_sel=None, order=None, status=None, head_dim_v=None,
+                    workspace=None):
+    """Top-k page selection per (request, KV head).  Returns (sel [B,Hkv,kmax], n_sel [B,Hkv]).
+
+    With ``workspace`` (from fused_workspace() for the same arguments) it calls
+    vt_select_pages_ws (the persistent kernel for GQA heads, B <= 2048)."""
     lib = load_library()
     kv = paged_kv(k_pool, v_pool, head_dim_v)
     a = decode_args(q, page_table, seq_lens, centroids, topk, bos, eos, 1.0, order, status)
@@ -193,6 +200,13 @@ def vt_select_pages(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bo
         sel = torch.empty((B, hkv, kmax), dtype=torch.int32, device=q.device)
     if n_sel is None:
         n_sel = torch.empty((B, hkv), dtype=torch.int32, device=q.device)
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8, contiguous=True)
+        rc = lib.vt_select_pages_ws(ctypes.byref(kv), ctypes.byref(a), sel.data_ptr(),
+                                    n_sel.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                    _stream(q))
+        _check(rc, "vt_select_pages_ws")
+        return sel, n_sel
     rc = lib.vt_select_pages(ctypes.byref(kv), ctypes.byref(a), sel.data_ptr(), n_sel.data_ptr(),
                              _stream(q))
     _check(rc, "vt_select_pages")
@@ -220,8 +234,11 @@ def vt_select_pages_approx(q, k_pool, v_pool, page_table, seq_lens, centroids, t
 
 
 def vt_sparse_decode(q, k_pool, v_pool, page_table, seq_lens, sel, n_sel, sm_scale, out=None,
-                     lse=None, status=None, head_dim_v=None, want_lse=True):
-    """Attention over a given page selection.  Returns (out [B,Hq,Dv] bf16, lse [B,Hq] or None)."""
+                     lse=None, status=None, head_dim_v=None, want_lse=True, workspace=None):
+    """Attention over a given page selection.  Returns (out [B,Hq,Dv] bf16, lse [B,Hq] or None).
+
+    With ``workspace`` (decode_workspace() for these arguments) it calls vt_sparse_decode_ws
+    (the persistent kernel for GQA heads, B <= 2048)."""
     lib = load_library()
     kv = paged_kv(k_pool, v_pool, head_dim_v)
     kmax = sel.shape[2]
@@ -231,10 +248,28 @@ def vt_sparse_decode(q, k_pool, v_pool, page_table, seq_lens, sel, n_sel, sm_sca
         out = torch.empty((B, hq, kv.head_dim_v), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8, contiguous=True)
+        rc = lib.vt_sparse_decode_ws(ctypes.byref(kv), ctypes.byref(a), sel.data_ptr(),
+                                     n_sel.data_ptr(), out.data_ptr(), _ptr(lse),
+                                     workspace.data_ptr(), workspace.numel(), _stream(q))
+        _check(rc, "vt_sparse_decode_ws")
+        return out, lse
     rc = lib.vt_sparse_decode(ctypes.byref(kv), ctypes.byref(a), sel.data_ptr(), n_sel.data_ptr(),
                               out.data_ptr(), _ptr(lse), _stream(q))
     _check(rc, "vt_sparse_decode")
     return out, lse
+
+
+def decode_workspace(q, k_pool, v_pool, page_table, seq_lens, sel, head_dim_v=None):
+    """A zeroed workspace for vt_sparse_decode(..., workspace=) with these arguments (the
+    decode call's arguments: kmax = sel.shape[2] selected pages, no centroids), or None."""
+    lib = load_library()
+    kv = paged_kv(k_pool, v_pool, head_dim_v)
+    kmax = sel.shape[2]
+    a = decode_args(q, page_table, seq_lens, None, kmax, 0, 0, 1.0, None, None)
+    n = int(lib.vt_fused_workspace_size(ctypes.byref(kv), ctypes.byref(a)))
+    return torch.zeros(n, dtype=torch.uint8, device=q.device) if n else None
 
 
 def vt_fused_workspace_size(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bos, eos,

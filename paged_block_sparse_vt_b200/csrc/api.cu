@@ -26,7 +26,7 @@ int mla_persist_max_batch();
 cudaError_t launch_mla_persist(const DecodeParams& p, int G, void* ws, int64_t unit_cap,
                                int sm_count, cudaStream_t s);
 cudaError_t launch_persist_fused(const DecodeParams& p, int D, int G, void* ws, int64_t unit_cap,
-                                 int sm_count, cudaStream_t s);
+                                 int sm_count, cudaStream_t s, int mode);
 }  // namespace vt
 
 using namespace vt;
@@ -206,7 +206,7 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
                             size_t ws_bytes, void* stream, int64_t unit_cap = 0,
                             bool approx = false, uint64_t seed = 0,
                             const int32_t* fill_pages = nullptr, int n_fill = 0,
-                            float* cent_out = nullptr) {
+                            float* cent_out = nullptr, bool split_on_persistent = false) {
   Shape sh;
   DecodeParams p;
   vt_status s = fill_params(kv, a, mode != kDecode, &sh, &p);
@@ -240,7 +240,11 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
   p.fill_pages = fill_pages;
   p.n_fill = n_fill;
   p.cent_out = cent_out;
-  if (mode == kFused && use_persistent(sh, a)) {
+  // the select-only and decode-only calls given a workspace run as modes of the persistent
+  // GQA kernel (the MLA form keeps its cluster kernels for them)
+  const bool persistent = use_persistent(sh, a) &&
+                          (mode == kFused || (split_on_persistent && sh.path == kPathGqa && ws));
+  if (persistent) {
     const size_t need = persist_bytes(sh, p, unit_cap);
     if (!ws || ws_bytes < need)
       return fail(VT_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need,
@@ -252,7 +256,7 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
     if (bytes > 227 * 1024) return fail(VT_ERR_UNSUPPORTED, "shared memory need %d B too large", bytes);
     cudaError_t e = sh.path == kPathMla
                         ? launch_mla_persist(p, sh.G, ws, unit_cap, sm_count(), st)
-                        : launch_persist_fused(p, sh.D, sh.G, ws, unit_cap, sm_count(), st);
+                        : launch_persist_fused(p, sh.D, sh.G, ws, unit_cap, sm_count(), st, mode);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return ok();
   }
@@ -325,6 +329,21 @@ vt_status vt_select_pages(const vt_paged_kv* kv, const vt_decode_args* a, int32_
   return launch_query_side(kv, a, kSelect, sel, n_sel, nullptr, nullptr, nullptr, 0, stream);
 }
 
+vt_status vt_select_pages_ws(const vt_paged_kv* kv, const vt_decode_args* a, int32_t* sel,
+                             int32_t* n_sel, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  return launch_query_side(kv, a, kSelect, sel, n_sel, nullptr, nullptr, workspace,
+                           workspace_bytes, stream, 0, false, 0, nullptr, 0, nullptr, true);
+}
+
+vt_status vt_sparse_decode_ws(const vt_paged_kv* kv, const vt_decode_args* a, const int32_t* sel,
+                              const int32_t* n_sel, void* out, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return launch_query_side(kv, a, kDecode, const_cast<int32_t*>(sel), const_cast<int32_t*>(n_sel),
+                           out, lse, workspace, workspace_bytes, stream, 0, false, 0, nullptr, 0,
+                           nullptr, true);
+}
+
 vt_status vt_select_pages_approx(const vt_paged_kv* kv, const vt_decode_args* a, uint64_t seed,
                                  int32_t* sel, int32_t* n_sel, void* stream) {
   return launch_query_side(kv, a, kSelect, sel, n_sel, nullptr, nullptr, nullptr, 0, stream, 0,
@@ -347,7 +366,7 @@ vt_status vt_sparse_decode_fused(const vt_paged_kv* kv, const vt_decode_args* a,
 size_t vt_fused_workspace_size(const vt_paged_kv* kv, const vt_decode_args* a) {
   Shape sh;
   DecodeParams p;
-  if (fill_params(kv, a, true, &sh, &p) != VT_OK) return 0;
+  if (fill_params(kv, a, false, &sh, &p) != VT_OK) return 0;  // (centroids are not needed)
   if (!use_persistent(sh, a)) return 0;
   return persist_bytes(sh, p, 0);
 }

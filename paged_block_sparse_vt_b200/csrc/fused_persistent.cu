@@ -102,6 +102,7 @@ struct PersistWs {
   int32_t* cpid;       // [U][nch_max][kc]: their page ids (-1 where the id was out of range)
   float* part;         // [U][A2][G][Dv+2]: attention partials
   PersistGeom g;
+  int mode;            // kFused, kSelect (scan items only) or kDecode (attention items only)
   int units;
 };
 
@@ -272,20 +273,40 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
     if (tid == 0) s_misc[0] = first;
     __syncthreads();
   }
-  const int scan_items = s_prefix[p.B];
+  const int scan_items = w.mode == kDecode ? 0 : s_prefix[p.B];
   // Units from u_split on take gm.A2 (shorter) pieces: only the attention that runs at the
   // end of the launch, where shorter items keep more CTAs busy, is split.  Measured: splitting
   // the last gridDim.x / 4 units (at least half of them) against the last half of the units:
   // 35.8 us both at the Qwen3-0.6B-like layer (256 units), 342 -> 324 us at 32K contexts
   // (1024 units), 260 -> 237 us on the heterogeneous batch (16384 units).
   const int u_split = max(w.units / 2, w.units - (int)gridDim.x / 4);
-  const int total_items = scan_items + u_split * gm.A + (w.units - u_split) * gm.A2;
+  const int total_items =
+      scan_items + (w.mode == kSelect ? 0 : u_split * gm.A + (w.units - u_split) * gm.A2);
+  if (w.mode == kSelect) {
+    // the units that rank nothing (dense, reserved only, or invalid): their selection here
+    for (int u = blockIdx.x; u < w.units; u += gridDim.x) {
+      const int b = u / p.Hkv;
+      const int L = p.seq_lens[b];
+      if (chunks_of(L, p.pt_stride, p.topk, p.bos, p.eos, p.kmax) > 0) continue;
+      const int n = (L + kPage - 1) / kPage;
+      const bool valid = L >= 1 && n <= p.pt_stride;
+      const int ns = !valid ? 0 : (n <= p.kmax ? n : p.kmax);
+      const bool resv = valid && n > p.kmax;
+      for (int j = tid; j < p.kmax; j += NT)
+        p.sel[(int64_t)u * p.kmax + j] =
+            j >= ns ? -1 : ((!resv || j < p.bos) ? j : n - p.eos + (j - p.bos));
+      if (tid == 0) {
+        p.n_sel[u] = ns;
+        if (!valid && u % p.Hkv == 0) flag(p.status, VT_DEV_BAD_LEN);
+      }
+    }
+  }
 
   // ---- scan items: where an item's rows lie, and its per-lane state.  A scan item whose
   // predecessor was a scan item finds its page ids and query mean already in registers and
   // its first kScanRing - 1 batches in flight (prepared during the predecessor's top-k).
   struct ScanItem {
-    int b, h, c, u, cnt, c0, myrows, batches;
+    int b, h, c, u, cnt, c0, myrows, batches, nch;
   };
   auto scan_item = [&](int t) {
     ScanItem it;
@@ -299,6 +320,7 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
     const int n = (p.seq_lens[it.b] + kPage - 1) / kPage;
     const int m = n - p.bos - p.eos;
     const int nch = (m + kChunk - 1) / kChunk;
+    it.nch = nch;
     it.h = r / nch;
     it.c = r - it.h * nch;
     it.u = it.b * p.Hkv + it.h;
@@ -365,6 +387,104 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
       }
     }
     cp_async_commit();
+  };
+  // ---- select-only launches: the unit's selection, taken by the CTA whose chunk was counted
+  // last for the unit: the exact top-k of the chunks' candidates (the union of the chunks'
+  // top-k holds the unit's top-k) plus the reserved pages, written to sel / n_sel in ascending
+  // logical order.
+  auto merge_unit = [&](int b, int u, int nch) {
+    const int n = (p.seq_lens[b] + kPage - 1) / kPage;
+    const int m = n - p.bos - p.eos;
+    const int kc = gm.kc;
+    const int C = (nch - 1) * kc + min(kc, m - (nch - 1) * kChunk);
+    const int64_t cb = (int64_t)u * gm.nch_max * kc;  // chunks are contiguous
+    const int bos = p.bos, topk = p.topk;
+    const int32_t* ptrow = p.page_table + (int64_t)b * p.pt_stride;
+    int32_t* selrow = p.sel + (int64_t)u * p.kmax;
+    if (tid == 0) p.n_sel[u] = p.kmax;
+    auto checked = [&](int pg) {
+      if (pg < 0 || pg >= p.num_pages) flag(p.status, VT_DEV_BAD_PAGE);
+    };
+    // the reserved pages (their page-id loads in flight with the candidates' loads)
+    const int nres = bos + p.eos;
+    int rlp = -1, rpg = -1;
+    if (tid < nres) {
+      rlp = tid < bos ? tid : n - p.eos + (tid - bos);
+      rpg = ptrow[rlp];
+    }
+    // candidate j of chunk j / kc sits at offset coff[j] of it; candidates are in ascending
+    // page order, so ties (lowest position) go to the lowest page
+    if (C <= 2 * NT) {
+      uint32_t* keys = reinterpret_cast<uint32_t*>(region);
+      int* lps = reinterpret_cast<int*>(region + 2 * NT * 4);
+      int* pids = reinterpret_cast<int*>(region + 4 * NT * 4);
+      unsigned char* tkm = region + 6 * NT * 4;
+      for (int i = tid; i < SmallTopk<NT>::HIST / 4; i += NT)
+        reinterpret_cast<int4*>(tkm)[i] = make_int4(0, 0, 0, 0);
+      const bool h0 = tid < C, h1 = tid + NT < C;
+      uint32_t key0 = 0, key1 = 0;
+      int off0 = 0, off1 = 0, pid0 = -1, pid1 = -1;
+      if (h0) {
+        key0 = __ldcg(w.ckey + cb + tid);
+        off0 = __ldcg(w.coff + cb + tid);
+        pid0 = __ldcg(w.cpid + cb + tid);
+      }
+      if (h1) {
+        key1 = __ldcg(w.ckey + cb + tid + NT);
+        off1 = __ldcg(w.coff + cb + tid + NT);
+        pid1 = __ldcg(w.cpid + cb + tid + NT);
+      }
+      uint32_t klo = 0xffffffffu, khi = 0u;
+      if (h0) {
+        keys[tid] = key0;
+        lps[tid] = bos + (tid / kc) * kChunk + off0;
+        pids[tid] = pid0;
+        klo = key0;
+        khi = key0;
+      }
+      if (h1) {
+        const int j = tid + NT;
+        keys[j] = key1;
+        lps[j] = bos + (j / kc) * kChunk + off1;
+        pids[j] = pid1;
+        klo = min(klo, key1);
+        khi = max(khi, key1);
+      }
+      klo = __reduce_min_sync(kFull, klo);
+      khi = __reduce_max_sync(kFull, khi);
+      if (lane == 0) {
+        s_misc[16 + warp] = (int)klo;
+        s_misc[16 + NW + warp] = (int)khi;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < NW; ++k) {
+        klo = min(klo, (uint32_t)s_misc[16 + k]);
+        khi = max(khi, (uint32_t)s_misc[16 + NW + k]);
+      }
+      small_topk<NT>(keys, C, topk, klo, khi, tkm, [&](int j, int pos) {
+        selrow[bos + pos] = lps[j];
+      });
+    } else {
+      uint32_t* keys = reinterpret_cast<uint32_t*>(region);
+      uint16_t* offs = reinterpret_cast<uint16_t*>(region + align16(gm.cmax * 4));
+      int* hist = reinterpret_cast<int*>(region + align16(gm.cmax * 4) + align16(gm.cmax * 2));
+      for (int j = tid; j < C; j += NT) {
+        keys[j] = __ldcg(w.ckey + cb + j);
+        offs[j] = __ldcg(w.coff + cb + j);
+      }
+      __syncthreads();
+      block_topk<NT>(keys, C, topk, hist, hist + kTopkBins, [&](int j, int pos) {
+        selrow[bos + pos] = bos + (j / kc) * kChunk + offs[j];
+      });
+    }
+    if (tid < nres) {
+      const int pos = tid < bos ? tid : bos + topk + (tid - bos);
+      checked(rpg);
+      selrow[pos] = rlp;
+    }
+    __syncthreads();
+    if (tid == 0) w.unit_done[u] = 0;  // every chunk of u is counted: the counter is free again
   };
   // scratch of a chunk's top-k: warp 0's last ring slot where it is large enough (the next
   // item's first batches fill the other slots meanwhile), else past the rings
@@ -487,7 +607,13 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
       // thread's stores before thread 0's release), then put the next chunk's first batches
       // in flight
       __syncthreads();
-      if (tid == 0) red_release_add(w.unit_done + it.u, 1);
+      if (w.mode == kSelect) {  // the chunk counted last for the unit takes its selection
+        if (tid == 0) s_misc[2] = atom_acq_rel_add(w.unit_done + it.u, 1) == it.nch - 1;
+        __syncthreads();
+        if (s_misc[2]) merge_unit(it.b, it.u, it.nch);
+      } else if (tid == 0) {
+        red_release_add(w.unit_done + it.u, 1);
+      }
       if (prepared) {
         scan_check(it2);
 #pragma unroll
@@ -505,15 +631,30 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
       const int n = (L + kPage - 1) / kPage;
       const bool valid = L >= 1 && n <= p.pt_stride;
       const bool dense = n <= p.kmax;
-      const int nch = chunks_of(L, p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
-      const int ns = !valid ? 0 : (dense ? n : p.kmax);
+      const bool dec = w.mode == kDecode;  // the selection is an input (sel, n_sel)
+      const int nch = dec ? 0 : chunks_of(L, p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
+      int ns = !valid ? 0 : (dense ? n : p.kmax);
+      if (dec) {
+        // every piece checks the unit's whole row, so that a bad entry anywhere zeroes all of
+        // the unit's outputs
+        const int nsi = valid ? p.n_sel[u] : 0;
+        int bad = valid && (nsi < 0 || nsi > p.kmax);
+        if (!bad)
+          for (int j = tid; j < nsi; j += NT) {
+            const int v = p.sel[(int64_t)u * p.kmax + j];
+            bad |= v < 0 || v >= n;
+          }
+        bad = __syncthreads_or(bad);
+        if (bad && tid == 0 && piece == 0) flag(p.status, VT_DEV_BAD_SEL);
+        ns = bad ? 0 : nsi;
+      }
       const int j0 = piece * pp;
       const int np = max(0, min(ns - j0, pp));
-      const bool write_sel = piece == 0 && p.sel != nullptr;
+      const bool write_sel = piece == 0 && p.sel != nullptr && !dec;
       int32_t* selrow = write_sel ? p.sel + (int64_t)u * p.kmax : nullptr;
       if (tid == 0 && piece == 0) {
         if (!valid && h == 0) flag(p.status, VT_DEV_BAD_LEN);
-        if (p.n_sel) p.n_sel[u] = ns;
+        if (p.n_sel && !dec) p.n_sel[u] = ns;
       }
       int ok = 1;
       if (nch > 0) {
@@ -657,12 +798,14 @@ __global__ void __launch_bounds__(kPersistThreads, kPersistMinCtas) persist_fuse
             });
           }
         } else {
-          // dense (every page, in order) or, with topk == 0, the reserved pages alone
+          // dense (every page, in order) or, with topk == 0, the reserved pages alone; or, in
+          // a decode-only launch, the given selection
           const bool resv = valid && !dense;
           auto page_at = [&](int pos) {
             return (!resv || pos < p.bos) ? pos : n - p.eos + (pos - p.bos);
           };
-          for (int q = tid; q < np; q += NT) s_sel[q] = page_at(j0 + q);
+          for (int q = tid; q < np; q += NT)
+            s_sel[q] = dec ? p.sel[(int64_t)u * p.kmax + j0 + q] : page_at(j0 + q);
           if (write_sel)
             for (int j = tid; j < p.kmax; j += NT) selrow[j] = j < ns ? page_at(j) : -1;
         }
@@ -830,7 +973,7 @@ static cudaError_t dispatch_persist_g(const DecodeParams& p, const PersistWs& w,
 // Launch the persistent kernel on `ws` (persist_workspace_bytes() bytes for the same
 // unit_cap, counters zero): as many CTAs as fit on the sm_count SMs at once.
 cudaError_t launch_persist_fused(const DecodeParams& p, int D, int G, void* ws, int64_t unit_cap,
-                                 int sm_count, cudaStream_t s) {
+                                 int sm_count, cudaStream_t s, int mode) {
   const PersistWsLayout L = persist_ws_layout(p, G, D, unit_cap);
   unsigned char* base = static_cast<unsigned char*>(ws);
   PersistWs w;
@@ -843,6 +986,7 @@ cudaError_t launch_persist_fused(const DecodeParams& p, int D, int G, void* ws, 
   w.part = reinterpret_cast<float*>(base + L.part);
   w.g = persist_geom(p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
   w.units = p.B * p.Hkv;
+  w.mode = mode;
   if (D == 64) return dispatch_persist_g<64>(p, w, G, sm_count, s);
   if (D == 128) return dispatch_persist_g<128>(p, w, G, sm_count, s);
   return cudaErrorInvalidValue;

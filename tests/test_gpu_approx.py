@@ -1,5 +1,6 @@
 """The indexer's lossy mode (vt_select_pages_approx) at the full sizes of the Qwen3-0.6B-like,
-long-context and heterogeneous workloads, against the oracle's lossy mode and its exact top-k.
+long-context, MLA latent and heterogeneous workloads, against the oracle's lossy mode and its
+exact top-k.
 
 Both sides decide the bins in fp32, but from scores rounded differently (the GPU's fp32 dot
 product, the oracle's fp64 one rounded once), so a candidate on a bin edge may fall on
@@ -22,7 +23,7 @@ MIN_SAME_FRACTION = 0.98   # units whose lossy set equals the oracle's lossy set
 MIN_RECALL, MIN_MEAN_RECALL = 0.90, 0.97
 
 
-@pytest.mark.parametrize("cfg", [2, 3, 5])
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
 def test_lossy_select_full_size(cfg, oracle):
     c = config(cfg)
     w = make_workload(c)
@@ -36,8 +37,8 @@ def test_lossy_select_full_size(cfg, oracle):
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     args = (d["q"], d["k_pool"], d["v_pool"], d["page_table"], d["seq_lens"], cent.cuda(),
             c.topk, c.bos, c.eos)
-    sel, n_sel = vt.vt_select_pages_approx(*args, seed, status=st)
-    sel2, _ = vt.vt_select_pages_approx(*args, seed)
+    sel, n_sel = vt.vt_select_pages_approx(*args, seed, status=st, head_dim_v=c.Dv)
+    sel2, _ = vt.vt_select_pages_approx(*args, seed, head_dim_v=c.Dv)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert torch.equal(sel, sel2)  # deterministic for a seed

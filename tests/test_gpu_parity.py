@@ -276,6 +276,15 @@ def test_bad_inputs_set_status_and_spare_other_units(oracle):
                         ref["n_sel"].cuda(), c.sm_scale, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == vt.VT_DEV_BAD_SEL
+    # the same through the decode-only persistent launch: reported, the unit's output zeroed
+    st.zero_()
+    ws = vt.decode_workspace(d["q"], d["k_pool"], d["v_pool"], d["page_table"], d["seq_lens"],
+                             bad_sel)
+    out, _ = vt.vt_sparse_decode(d["q"], d["k_pool"], d["v_pool"], d["page_table"], d["seq_lens"],
+                                 bad_sel, ref["n_sel"].cuda(), c.sm_scale, status=st, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(st.item()) == vt.VT_DEV_BAD_SEL
+    assert torch.all(out[2, :c.G].float() == 0)
 
 
 @pytest.mark.parametrize("name", ["c2s", "c4s", "c5s"])
@@ -309,3 +318,31 @@ def test_last_page_centroid_is_never_read(name):
         res.append((out.view(torch.int16), lse, sel, n_sel))
     for a, b in zip(*res):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_select_and_decode_with_workspace(name, oracle):
+    """vt_select_pages_ws and vt_sparse_decode_ws (the persistent kernel's select-only and
+    decode-only launches for GQA heads, B <= 2048; the other shapes keep the cluster kernels)
+    against the oracle, twice in a row on the same workspaces."""
+    w = _case(name)
+    c = w["config"]
+    d = to_device(w)
+    cent_ref, ref = _reference(name)
+    cent = cent_ref.cuda()
+    args = (d["q"], d["k_pool"], d["v_pool"], d["page_table"], d["seq_lens"], cent, c.topk, c.bos,
+            c.eos)
+    ws_sel = vt.fused_workspace(*args, head_dim_v=c.Dv)
+    ref_sel, ref_n = ref["sel"].cuda(), ref["n_sel"].cuda()
+    ws_dec = vt.decode_workspace(d["q"], d["k_pool"], d["v_pool"], d["page_table"], d["seq_lens"],
+                                 ref_sel, head_dim_v=c.Dv)
+    for _ in range(2):
+        st = _status()
+        sel, n_sel = vt.vt_select_pages(*args, status=st, head_dim_v=c.Dv, workspace=ws_sel)
+        out, lse = vt.vt_sparse_decode(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                       d["seq_lens"], ref_sel, ref_n, c.sm_scale, status=st,
+                                       head_dim_v=c.Dv, workspace=ws_dec)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        compare_selection(w, ref, cent_ref, sel, n_sel, label=f"select with workspace {name}")
+        compare_outputs(out, lse, ref["out"], ref["lse"])
