@@ -10,26 +10,29 @@
 // q_lat . c_lat + q_rope . c_rope is one dot product over the 576-dim row (the page mean is
 // linear in each part).
 //
-// One CTA of 8 warps per SM (the attention stages Q and two buffers of four K tiles: ~200 KB).
+// One CTA of 8 warps per SM (two K tiles, Q, P and the round's scores: ~208 KB of shared
+// memory; 256 columns of tensor memory held for the whole launch).
 // Items:
 //   build items  -- (vt_sparse_decode_step only) the centroid of one page filled at this step;
 //   scan items   -- (request, chunk of kMlaChunk candidate pages): each warp streams its rows
 //                   of fp32 centroids (2304 B each) through a cp.async ring and dots them with
 //                   the fp32 mean of the request's query heads; the CTA keeps the chunk's exact
 //                   top-k (key, offset, page id) and counts the chunk done;
-//   attention    -- (request, piece of <= kMpPiece selected pages): waits until every chunk of
-//   items           the request is counted, merges the chunks' candidates with the same exact
-//                   top-k, then takes the piece's pages in rounds of kMpRound: their K tiles
-//                   land in one buffer while the previous round computes from the other;
-//                   S^T = K Q^T (two warps per page, 16 heads each), the softmax against each
-//                   head's running maximum, and O = P V (each warp owns 64 of the 512 output
-//                   dims, rescaled when the maximum moves) on the tensor cores; with several
-//                   pieces, the last one waits for the others' partials in the workspace and
-//                   merges them in registers.
+//   attention    -- (request, piece of the selected pages): waits until every chunk of the
+//   items           request is counted, merges the chunks' candidates with the same exact
+//                   top-k, then takes the piece's pages in rounds of kMpRound on the fifth-
+//                   generation tensor cores: S^T = K Q^T (M = 64 tokens, N = G heads) and
+//                   O^T += V^T P^T (M = 128 output dims, N = G) with both accumulators in
+//                   tensor memory, the operands in 128-byte swizzled shared memory (V^T is the
+//                   K tile read MN-major), an online softmax between them, and one K tile
+//                   landing while the other round computes.  With several pieces, the earlier
+//                   ones take whole rounds and publish fp32 partials with one bulk copy each;
+//                   the last piece folds them in and writes the request's rows.
 // Queue, claims and counters work as in the GQA persistent kernel (fused_persistent.cu).
 #include "centroid_chunk.cuh"
 #include "decode_params.cuh"
 #include "topk.cuh"
+#include "umma.cuh"
 
 namespace vt {
 
@@ -37,12 +40,16 @@ constexpr int kMpThreads = 256;
 constexpr int kMpWarps = kMpThreads / 32;
 constexpr int kMpD = 576;
 constexpr int kMpDv = 512;
-constexpr int kMpRow = kMpD + 8;   // smem row stride of Q and K tiles (elements): conflict-free ldmatrix
 constexpr int kMlaChunk = 256;     // candidate pages per scan item (32 per warp)
 constexpr int kMpScanRows = 2;     // centroid rows per ring slot
 constexpr int kMpScanSlots = 5;    // ring slots per warp (4 landing while one is used)
-constexpr int kMpPiece = 32;       // most selected pages per attention item
+constexpr int kMpPiece = 32;       // selected pages per attention item (target)
 constexpr int kMpRound = 4;        // pages of a piece staged and computed together (64 tokens)
+constexpr int kMpKtBytes = (kMpD / 64) * kMpRound * kPage * 128;  // one round's K tile (72 KB)
+constexpr int kMpOcol = 64;        // tensor-memory column of O^T (S^T buffers take [0, 2G))
+constexpr int kMpTmemCols = 256;   // tensor-memory columns a CTA holds: 2 G + 4 G <= 192
+constexpr int kMpSelCap = kMpPiece + kMpRound;  // most pages of one piece (the last one)
+constexpr float kLazyRescale = 8.0f;  // base-2 growth of a head's maximum that moves its reference
 constexpr int kMpMaxB = 2048;      // requests the persistent path takes
 
 // ---- sizes derived from the call ----------------------------------------------------------
@@ -52,7 +59,7 @@ struct MpGeom {
   int nch_max;   // chunks of such a row
   int kc;        // candidates a chunk keeps: min(topk, kMlaChunk)
   int cmax;      // candidates one request merges at most
-  int A, pp;     // attention pieces per request and their selected pages
+  int A, pp;     // attention pieces per request, pages of each but the last (which takes the rest)
 };
 
 __host__ __device__ inline MpGeom mp_geom(int64_t pt_stride, int topk, int bos, int eos, int kmax) {
@@ -65,6 +72,12 @@ __host__ __device__ inline MpGeom mp_geom(int64_t pt_stride, int topk, int bos, 
   g.cmax = c < g.max_cand ? (int)c : g.max_cand;
   g.A = (kmax + kMpPiece - 1) / kMpPiece;
   g.pp = (kmax + g.A - 1) / g.A;
+  // the pieces before the last take whole rounds, so that they publish their partials about a
+  // round before the last piece (which merges them) finishes its own pages
+  if (g.A > 1) {
+    const int pr = (g.pp / kMpRound) * kMpRound;
+    if (pr >= kMpRound && kmax - (g.A - 1) * pr <= kMpSelCap) g.pp = pr;
+  }
   return g;
 }
 
@@ -114,9 +127,9 @@ static MpWsLayout mp_ws_layout(const DecodeParams& p, int G, int64_t unit_cap) {
 // ---- shared memory -------------------------------------------------------------------------
 
 struct MpSmem {
-  int prefix, keys, pids, qm, sel, phys, ml, misc, region;  // region: one phase at a time
-  int ring, q, kt, pm, pmax, psum, fac;                     // region offsets
-  int total;
+  int prefix, keys, pids, qm, sel, phys, ml, misc, tc, region;  // region: one phase at a time
+  int ring, q, kt, pb, sc, fac, mm;                             // region offsets
+  int total;  // including 1 KB to align the base to the 1024-byte swizzle atoms
 };
 
 __host__ __device__ inline MpSmem mp_smem_layout(int G, int B, const MpGeom& g) {
@@ -126,11 +139,12 @@ __host__ __device__ inline MpSmem mp_smem_layout(int G, int B, const MpGeom& g) 
   s.keys = o;   o += align16(kMlaChunk * 4);
   s.pids = o;   o += align16(kMlaChunk * 4);
   s.qm = o;     o += align16(kMpD * 4);
-  s.sel = o;    o += align16(kMpPiece * 4);
-  s.phys = o;   o += align16(kMpPiece * 4);
+  s.sel = o;    o += align16(kMpSelCap * 4);
+  s.phys = o;   o += align16(kMpSelCap * 4);
   s.ml = o;     o += align16(G * 2 * 4);
   s.misc = o;   o += align16(64 * 4);
-  o = (o + 127) & ~127;
+  s.tc = o;     o += 64;  // three mbarriers, the tensor-memory address
+  o = (o + 1023) & ~1023;
   s.region = o;
   // scan: per-warp rings of centroid rows (the chunk top-k scratch reuses warp 0's ring)
   s.ring = 0;
@@ -140,19 +154,20 @@ __host__ __device__ inline MpSmem mp_smem_layout(int G, int B, const MpGeom& g) 
   const int merge_big = align16(g.cmax * 4) + align16(g.cmax * 2) + align16((kTopkBins + 64) * 4);
   const int merge = merge_small > merge_big ? merge_small : merge_big;
   // attention: two buffers of a round's K tiles (first: the merge scratch above is dead once
-  // they load), Q (prefetched while the merge runs), P, per-page maxima and sums, rescales
+  // they load), Q (prefetched while the merge runs), two P buffers, the round's scores,
+  // rescale factors, the merge's per-head factors; the swizzled operands on 1024-byte bounds
   const int RT = kMpRound * kPage;
   int a = 0;
-  s.kt = a; a += align16(2 * RT * kMpRow * 2);
-  s.q = a;  a += align16(G * kMpRow * 2);
-  s.pm = a; a += align16(G * (RT + 8) * 2);
-  s.pmax = a; a += align16(kMpRound * G * 4);
-  s.psum = a; a += align16(kMpRound * G * 4);
+  s.kt = a; a += 2 * kMpKtBytes;
+  s.q = a;  a += (kMpD / 64) * G * 128;
+  s.pb = a; a += 2 * G * 128;
+  s.sc = a; a += G * RT * 4;
   s.fac = a; a += align16(G * 4);
+  s.mm = a; a += align16(G * 4 * 4);
   int r = scan;
   if (merge > r) r = merge;
   if (a > r) r = a;
-  s.total = o + r;
+  s.total = o + r + 1024;
   return s;
 }
 
@@ -187,15 +202,21 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
   constexpr int CH4 = D / 4;  // float4 per centroid row
   constexpr int RB = D * 4;   // bytes of a centroid row
   constexpr int RT = kMpRound * kPage;  // tokens of a round
-  constexpr int PST = RT + 8;
   static_assert(G == 16 || G == 32, "MLA path covers 16 or 32 query heads");
   static_assert(kMlaChunk <= 32 * kMpWarps, "one page id per lane: at most 32 rows per warp");
-  static_assert(kMpRound >= 2, "the page-max table [kMpRound][G] holds the merge's [G][2]");
-  static_assert(kMpRound * 2 <= kMpWarps, "S^T: a warp per page of a round (two when G = 32)");
+  static_assert(RT == 64, "S^T is one M = 64 tile per round: four warps of 16 tokens");
+  static_assert(kMpWarps == 8 && DV == 512, "O^T: eight warps hold 2 of its 4 blocks each");
+  static_assert(kMpOcol >= 2 * G && kMpOcol + 4 * G <= kMpTmemCols, "tensor-memory columns");
   static_assert(SmallTopk<NT>::BYTES <= kMpScanSlots * kMpScanRows * RB,
                 "the chunk top-k scratch fits in warp 0's ring");
+  // S^T: M = 64 tokens x N = G heads, both operands K-major; O^T: M = 128 dims x N = G heads,
+  // A (V^T) MN-major, B (P) K-major
+  constexpr uint32_t kIdescS = umma::idesc_bf16(64, G, false, false);
+  constexpr uint32_t kIdescO = umma::idesc_bf16(128, G, true, false);
 
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // the swizzle atoms need 1024-byte alignment in the shared window
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const MpGeom gm = w.g;
   const MpSmem Ls = mp_smem_layout(G, p.B, gm);
   int* s_prefix = reinterpret_cast<int*>(smem + Ls.prefix);
@@ -213,6 +234,39 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
   // programmatic dependent launch: nothing global is touched before the previous kernel ends
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+
+  // tensor memory for the whole launch (warp 0), and the mbarriers: [0], [1] S^T of even and
+  // odd rounds, [2] O^T, [3] a partial's bulk load.  Each completion is waited on exactly
+  // once, by every thread, so the phase bits below stay in step.
+  const uint32_t bars_a = smem_u32(smem + Ls.tc);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Ls.tc + 32);
+  if (warp == 0) umma::tmem_alloc(smem_u32(s_tmem), kMpTmemCols);
+  if (tid == 0) {
+    umma::mbar_init(bars_a, 1);
+    umma::mbar_init(bars_a + 8, 1);
+    umma::mbar_init(bars_a + 16, 1);
+    umma::mbar_init(bars_a + 24, 1);
+    umma::mbar_fence_init();
+  }
+  umma::fence_before_sync();
+  __syncthreads();
+  umma::fence_after_sync();
+  const uint32_t tm = *s_tmem;
+  uint32_t phases = 0u;  // bit i: the parity of mbarrier i's next completion
+  // bounded wait for the next completion of mbarrier `which`
+  auto bar_wait = [&](int which) {
+    const uint32_t bar = bars_a + 8 * which, ph = (phases >> which) & 1u;
+    if (!umma::mbar_try_wait(bar, ph)) {
+      const unsigned long long t0 = global_ns();
+      while (!umma::mbar_try_wait(bar, ph)) {
+        if (global_ns() - t0 > kWaitNs) {
+          flag(p.status, kDevTimeout);
+          break;
+        }
+      }
+    }
+    phases ^= 1u << which;
+  };
 
   uint32_t qbase = 0;  // thread 0: the claim count when this launch began
   // items are numbered from -n_fill: the build items of the pages filled at this step first
@@ -492,7 +546,7 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
       const int nch = mp_chunks(L, p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
       const int ns = !valid ? 0 : (dense ? n : p.kmax);
       const int j0 = piece * ppb;
-      const int np = max(0, min(ns - j0, ppb));
+      const int np = piece == Ab - 1 ? max(0, ns - j0) : max(0, min(ns - j0, ppb));
       const bool write_sel = piece == 0 && p.sel != nullptr;
       int32_t* selrow = write_sel ? p.sel + (int64_t)b * p.kmax : nullptr;
       const int64_t orow = (int64_t)b * p.Hq;
@@ -506,11 +560,12 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
       const int m_c = n - p.bos - p.eos;
       const int C_c = nch > 0 ? (nch - 1) * gm.kc + min(gm.kc, m_c - (nch - 1) * kMlaChunk) : 0;
       const bool q_early = C_c <= 2 * NT;
-      __nv_bfloat16* s_q = reinterpret_cast<__nv_bfloat16*>(region + Ls.q);
+      const uint32_t q_a = smem_u32(region + Ls.q);  // [atom][G rows][128 B], swizzled K-major
       auto stage_q = [&]() {
         for (int i = tid; i < G * (D / 8); i += NT) {
           const int g = i / (D / 8), c8 = i - g * (D / 8);
-          cp_async16(smem_u32(s_q + g * kMpRow + c8 * 8), p.q + (orow + g) * D + c8 * 8, 16);
+          cp_async16(q_a + (c8 >> 3) * (G * 128) + umma::sw128_off(g, c8 & 7),
+                     p.q + (orow + g) * D + c8 * 8, 16);
         }
         cp_async_commit();
       };
@@ -625,279 +680,307 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
           if (tid < np) s_phys[tid] = phys_of(s_sel[tid]);
           __syncthreads();
         }
-        // ---- the piece's pages in rounds of kMpRound: K tiles (zero rows past the valid
-        // tokens) double-buffered, so that round r + 1 lands while round r computes; an online
-        // softmax carries each head's running maximum and sum from round to round
-        __nv_bfloat16* s_kt = reinterpret_cast<__nv_bfloat16*>(region + Ls.kt);  // [2][RT][kMpRow]
-        __nv_bfloat16* s_pm = reinterpret_cast<__nv_bfloat16*>(region + Ls.pm);  // [G][RT+8]
-        float* s_pmax = reinterpret_cast<float*>(region + Ls.pmax);             // [round page][G]
-        float* s_psum = reinterpret_cast<float*>(region + Ls.psum);             // [round page][G]
-        float* s_fac = reinterpret_cast<float*>(region + Ls.fac);               // [G]
-        float* s_run = s_ml;                                                     // [G][2]
+        // ---- the piece's pages in rounds of kMpRound pages (RT = 64 tokens) on the tensor cores.
+        // A round's K tile lands (zero rows past the valid tokens) in 128-byte swizzled K-major
+        // order in one of two buffers; per round
+        //   S^T = K Q^T      M = 64 tokens, N = G heads, K = 576, into tensor memory;
+        //   the softmax of each head against its reference maximum, through a shared-memory
+        //                    transpose of S^T (a group of NT / G threads per head); P in bf16,
+        //                    heads x tokens, as the next MMA's K-major operand;
+        //   O^T += V^T P^T   M = 128 output dims per block (four blocks), N = G, K = the round's
+        //                    tokens; V^T is the latent part of the same K tile, read MN-major;
+        //                    O^T stays in tensor memory for the whole piece.
+        // A head's reference maximum moves only when a round's maximum exceeds it by more than
+        // kLazyRescale (base 2), and O^T is then rescaled in tensor memory; P stays below 2^8.
+        // The tensor core runs round r's MMAs while round r + 1's tile lands in the other buffer.
+        unsigned char* kt = region + Ls.kt;
+        const uint32_t kt_a = smem_u32(kt), pb_a = smem_u32(region + Ls.pb);
+        float* s_sc = reinterpret_cast<float*>(region + Ls.sc);    // [G][RT] scores of the round
+        float* s_fac = reinterpret_cast<float*>(region + Ls.fac);  // [G] rescale factors
         const int last_valid = L - kPage * (n - 1);
         if (!q_early) stage_q();
         const int nr = (np + kMpRound - 1) / kMpRound;
         auto row_ok = [&](int j, int tt) {  // token tt of the piece's j-th page is attended
           return j < np && s_phys[j] >= 0 && (s_sel[j] != n - 1 || tt < last_valid);
         };
+        // staging: thread t copies rows t / 8 and t / 8 + 32 of the round, 16-byte chunk t % 8
+        // of each of the nine 128-byte atoms (eight threads read 128 contiguous bytes of a row)
+        static_assert(NT == 4 * RT, "eight threads per row, two rows per thread");
+        const int st_c = tid & 7;
         auto stage_round = [&](int r) {  // every thread commits one group per call
           if (r < nr) {
-            __nv_bfloat16* dst = s_kt + (r & 1) * RT * kMpRow;
-            constexpr int C8 = D / 8;  // 16-byte chunks per K row
-            for (int i = tid; i < RT * C8; i += NT) {
-              const int row = i / C8, c8 = i - row * C8;
+            const uint32_t buf = kt_a + (r & 1) * kMpKtBytes;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int row = (tid >> 3) + 32 * h2;
               const int j = r * kMpRound + row / kPage, tt = row % kPage;
               const bool ok_row = row_ok(j, tt);
               const __nv_bfloat16* src =
-                  ok_row ? p.k_pool + (int64_t)s_phys[j] * p.sk_p + (int64_t)tt * p.sk_t + c8 * 8
+                  ok_row ? p.k_pool + (int64_t)s_phys[j] * p.sk_p + (int64_t)tt * p.sk_t + st_c * 8
                          : p.k_pool;
-              cp_async16(smem_u32(dst + row * kMpRow + c8 * 8), src, ok_row ? 16 : 0);
+              const uint32_t dst = buf + umma::sw128_off(row, st_c);
+#pragma unroll
+              for (int kb = 0; kb < D / 64; ++kb)
+                cp_async16(dst + kb * (RT * 128), src + (ok_row ? kb * 64 : 0), ok_row ? 16 : 0);
             }
           }
           cp_async_commit();
         };
+        constexpr int TPH = NT / G;   // softmax threads per head
+        constexpr int TPT = RT / TPH; // tokens per softmax thread
+        const int sh = tid / TPH, spart = tid % TPH;  // this thread's head and token group
+        float M_run = -INFINITY, L_run = 0.0f;        // the head's reference maximum and sum
         stage_round(0);
         stage_round(1);
-        for (int g = tid; g < G; g += NT) {
-          s_run[2 * g] = -INFINITY;
-          s_run[2 * g + 1] = 0.0f;
-        }
-        float oacc[G / 16][8][4];
-#pragma unroll
-        for (int mt = 0; mt < G / 16; ++mt)
-#pragma unroll
-          for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) oacc[mt][nt][i] = 0.0f;
-        // S^T: warp w takes page w % kMpRound of the round and 16 of the heads (the second
-        // half of them on warps kMpRound.. when G = 32); its lane holds tokens r0 = lane/4
-        // and r0 + 8, heads hb + nt*8 + 2 (lane%4) + {0, 1}
-        constexpr int SPLIT = G / 16;  // warps per page in S^T
-        const int spage = warp % kMpRound, hb = (warp / kMpRound) * 16;
-        const bool s_warp = warp < kMpRound * SPLIT;
-        const int r0 = lane >> 2;
         for (int r = 0; r < nr; ++r) {
-          cp_async_wait<1>();  // this thread's share of round r (and of Q) has landed
-          __syncthreads();     // everyone's has; the running statistics are initialised
-          const __nv_bfloat16* kt = s_kt + (r & 1) * RT * kMpRow;
-          const int j = r * kMpRound + spage;  // the piece's page this warp scores
-          float acc[2][4];
+          // round r has landed (and Q with it): S^T(r) on the tensor core
+          if (r == 0) cp_async_wait<1>(); else cp_async_wait<0>();
+          umma::fence_async_smem();
+          __syncthreads();
+          if (warp == 0) {
+            umma::fence_after_sync();
+            const uint32_t ka = kt_a + (r & 1) * kMpKtBytes;
+            const uint32_t d = tm + (uint32_t)((r & 1) * G);
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
-          if (s_warp && j < np) {
-            const uint32_t a_base =
-                smem_u32(kt + (spage * 16 + (lane & 15)) * kMpRow + (lane >> 4) * 8);
-            const uint32_t b_base = smem_u32(
-                s_q + (hb + (lane & 7) + ((lane >> 4) << 3)) * kMpRow + ((lane >> 3) & 1) * 8);
-#pragma unroll 4
-            for (int ks = 0; ks < D / 16; ++ks) {
-              uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-              ldsm_x4(a_base + ks * 32, a0, a1, a2, a3);
-              ldsm_x4(b_base + ks * 32, b0, b1, b2, b3);
-              mma_16816(acc[0], a0, a1, a2, a3, b0, b1);
-              mma_16816(acc[1], a0, a1, a2, a3, b2, b3);
-            }
+            for (int ks = 0; ks < D / 16; ++ks)
+              umma::mma_bf16(d, umma::sdesc_sw128(ka + (ks >> 2) * (RT * 128) + (ks & 3) * 32, 16, 1024),
+                             umma::sdesc_sw128(q_a + (ks >> 2) * (G * 128) + (ks & 3) * 32, 16, 1024),
+                             kIdescS, ks > 0 ? 1u : 0u);
+            umma::commit(bars_a + 8 * (r & 1));
           }
-          // page maxima per head (base 2, masked tokens -inf)
-          const bool v0 = s_warp && row_ok(j, r0), v1 = s_warp && row_ok(j, r0 + 8);
+          if (r >= 1) {
+            // O^T(r - 1) has completed (its commit is waited on once), so the buffer it read
+            // takes round r + 1
+            bar_wait(2);
+            if (r + 1 < nr) stage_round(r + 1);
+          }
+          bar_wait(r & 1);
+          umma::fence_after_sync();
+          if (warp < 4) {  // token 16 w + lane (lane < 16) sits in lane 32 w + lane
+            uint32_t v[G / 16][16];
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            acc[nt][0] = v0 ? acc[nt][0] * p.qscale : -INFINITY;
-            acc[nt][1] = v0 ? acc[nt][1] * p.qscale : -INFINITY;
-            acc[nt][2] = v1 ? acc[nt][2] * p.qscale : -INFINITY;
-            acc[nt][3] = v1 ? acc[nt][3] * p.qscale : -INFINITY;
-            float m0 = fmaxf(acc[nt][0], acc[nt][2]), m1 = fmaxf(acc[nt][1], acc[nt][3]);
+            for (int c = 0; c < G / 16; ++c)
+              umma::tmem_ld16(tm + ((uint32_t)(32 * warp) << 16) + (uint32_t)((r & 1) * G + 16 * c), v[c]);
+            umma::fence_before_sync();
+            if (lane < 16) {
+              const bool ok = row_ok(r * kMpRound + warp, lane);
+              const int t = 16 * warp + lane;
 #pragma unroll
-            for (int o = 4; o <= 16; o <<= 1) {
-              m0 = fmaxf(m0, __shfl_xor_sync(kFull, m0, o));
-              m1 = fmaxf(m1, __shfl_xor_sync(kFull, m1, o));
-            }
-            if (s_warp && lane < 4) {
-              s_pmax[spage * G + hb + nt * 8 + 2 * lane] = m0;
-              s_pmax[spage * G + hb + nt * 8 + 2 * lane + 1] = m1;
+              for (int h = 0; h < G; ++h)
+                s_sc[h * RT + t] = ok ? __uint_as_float(v[h >> 4][h & 15]) * p.qscale : -INFINITY;
             }
           }
           __syncthreads();
-          // probabilities against the new running maximum (rounded once to bf16, as the P V
-          // MMA reads them) and their sums per page and head
-          if (s_warp) {
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-              const int c = hb + nt * 8 + 2 * (lane & 3);
-              float M0 = s_run[2 * c], M1 = s_run[2 * (c + 1)];
-#pragma unroll
-              for (int q = 0; q < kMpRound; ++q) {
-                M0 = fmaxf(M0, s_pmax[q * G + c]);
-                M1 = fmaxf(M1, s_pmax[q * G + c + 1]);
-              }
-              const __nv_bfloat16 p00 = __float2bfloat16(acc[nt][0] == -INFINITY ? 0.0f : exp2f(acc[nt][0] - M0));
-              const __nv_bfloat16 p01 = __float2bfloat16(acc[nt][1] == -INFINITY ? 0.0f : exp2f(acc[nt][1] - M1));
-              const __nv_bfloat16 p10 = __float2bfloat16(acc[nt][2] == -INFINITY ? 0.0f : exp2f(acc[nt][2] - M0));
-              const __nv_bfloat16 p11 = __float2bfloat16(acc[nt][3] == -INFINITY ? 0.0f : exp2f(acc[nt][3] - M1));
-              const int tk = spage * 16 + r0;
-              s_pm[c * PST + tk] = p00;
-              s_pm[(c + 1) * PST + tk] = p01;
-              s_pm[c * PST + tk + 8] = p10;
-              s_pm[(c + 1) * PST + tk + 8] = p11;
-              // the sums use the rounded weights, as the MMA does
-              float l0 = __bfloat162float(p00) + __bfloat162float(p10);
-              float l1 = __bfloat162float(p01) + __bfloat162float(p11);
-#pragma unroll
-              for (int o = 4; o <= 16; o <<= 1) {
-                l0 += __shfl_xor_sync(kFull, l0, o);
-                l1 += __shfl_xor_sync(kFull, l1, o);
-              }
-              if (lane < 4) {
-                s_psum[spage * G + c] = l0;
-                s_psum[spage * G + c + 1] = l1;
-              }
-            }
-          }
-          __syncthreads();
-          // the running statistics move to the new maximum; O is rescaled by s_fac below
-          for (int g = tid; g < G; g += NT) {
-            const float Mo = s_run[2 * g];
-            float Mn = Mo, Ls = 0.0f;
-            for (int q = 0; q < kMpRound; ++q) {
-              Mn = fmaxf(Mn, s_pmax[q * G + g]);
-              Ls += s_psum[q * G + g];
-            }
-            const float f = (Mo == -INFINITY) ? 0.0f : exp2f(Mo - Mn);
-            s_fac[g] = f;
-            s_run[2 * g] = Mn;
-            s_run[2 * g + 1] = fmaf(s_run[2 * g + 1], f, Ls);
-          }
-          __syncthreads();
-          // O += P V over the round's tokens: warp w owns output dims [64 w, 64 w + 64) for
-          // all G heads; V is the first 512 dims of the staged K rows
-#pragma unroll
-          for (int mt = 0; mt < G / 16; ++mt)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const float f = s_fac[mt * 16 + (lane >> 2) + 8 * hh];
-#pragma unroll
-              for (int nt = 0; nt < 8; ++nt) {
-                oacc[mt][nt][2 * hh] *= f;
-                oacc[mt][nt][2 * hh + 1] *= f;
-              }
-            }
+          // softmax of head sh over tokens [TPT spart, TPT spart + TPT) of the round
+          int need = 0;
           {
-            const int pr = min(kMpRound, np - r * kMpRound);  // pages of this round
-            const uint32_t pa_base = smem_u32(s_pm + (lane & 15) * PST + (lane >> 4) * 8);
-            const uint32_t vb_base = smem_u32(kt + ((lane & 7) + ((lane >> 3) & 1) * 8) * kMpRow +
-                                              warp * 64 + (lane >> 4) * 8);
-            for (int ks = 0; ks < pr; ++ks) {  // 16 tokens per step
-              uint32_t ar[G / 16][4];
+            float sv[TPT];
 #pragma unroll
-              for (int mt = 0; mt < G / 16; ++mt)
-                ldsm_x4(pa_base + (mt * 16 * PST + ks * 16) * 2, ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3]);
-#pragma unroll
-              for (int n2 = 0; n2 < 4; ++n2) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(vb_base + (ks * 16 * kMpRow + n2 * 16) * 2, b0, b1, b2, b3);
-#pragma unroll
-                for (int mt = 0; mt < G / 16; ++mt) {
-                  mma_16816(oacc[mt][2 * n2], ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3], b0, b1);
-                  mma_16816(oacc[mt][2 * n2 + 1], ar[mt][0], ar[mt][1], ar[mt][2], ar[mt][3], b2, b3);
-                }
-              }
+            for (int i = 0; i < TPT; i += 4) {
+              const float4 f4 = *reinterpret_cast<const float4*>(s_sc + sh * RT + spart * TPT + i);
+              sv[i] = f4.x; sv[i + 1] = f4.y; sv[i + 2] = f4.z; sv[i + 3] = f4.w;
             }
+            float mr = sv[0];
+#pragma unroll
+            for (int i = 1; i < TPT; ++i) mr = fmaxf(mr, sv[i]);
+#pragma unroll
+            for (int o = 1; o < TPH; o <<= 1) mr = fmaxf(mr, __shfl_xor_sync(kFull, mr, o));
+            const float Mn = mr > M_run + kLazyRescale ? mr : M_run;
+            const float fac = Mn == M_run ? 1.0f : (M_run == -INFINITY ? 0.0f : exp2f(M_run - Mn));
+            float ls = 0.0f;
+            uint32_t pk[TPT / 2];
+#pragma unroll
+            for (int i = 0; i < TPT; i += 2) {
+              const __nv_bfloat16 p0 = __float2bfloat16(sv[i] == -INFINITY ? 0.0f : exp2f(sv[i] - Mn));
+              const __nv_bfloat16 p1 = __float2bfloat16(sv[i + 1] == -INFINITY ? 0.0f : exp2f(sv[i + 1] - Mn));
+              ls += __bfloat162float(p0) + __bfloat162float(p1);  // the weights the MMA reads
+              pk[i / 2] = (uint32_t)__bfloat16_as_ushort(p0) | ((uint32_t)__bfloat16_as_ushort(p1) << 16);
+            }
+#pragma unroll
+            for (int o = 1; o < TPH; o <<= 1) ls += __shfl_xor_sync(kFull, ls, o);
+            L_run = fmaf(L_run, fac, ls);
+            M_run = Mn;
+            unsigned char* prow = region + Ls.pb + (r & 1) * (G * 128);
+            if constexpr (TPT == 8) {
+              *reinterpret_cast<uint4*>(prow + umma::sw128_off(sh, spart)) =
+                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            } else {
+              *reinterpret_cast<uint2*>(prow + umma::sw128_off(sh, spart >> 1) + (spart & 1) * 8) =
+                  make_uint2(pk[0], pk[1]);
+            }
+            if (spart == 0) s_fac[sh] = fac;
+            need = (r > 0 && fac != 1.0f) ? 1 : 0;
           }
-          __syncthreads();  // every warp is done with this buffer and with P
-          stage_round(r + 2);
+          umma::fence_async_smem();  // P is read by the tensor core
+          if (__syncthreads_or(need)) {
+            // O^T *= fac per head (column); O^T(r - 1) has completed.  Warp w rescales blocks
+            // 2 (w / 4) and 2 (w / 4) + 1 in its lane quarter.
+            const int sp = warp & 3, bh = warp >> 2;
+#pragma unroll
+            for (int bi = 0; bi < 2; ++bi)
+#pragma unroll
+              for (int c = 0; c < G / 16; ++c) {
+                const uint32_t ta = tm + ((uint32_t)(32 * sp) << 16) +
+                                    (uint32_t)(kMpOcol + G * (2 * bh + bi) + 16 * c);
+                uint32_t v[16];
+                umma::tmem_ld16(ta, v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                  v[j] = __float_as_uint(__uint_as_float(v[j]) * s_fac[16 * c + j]);
+                umma::tmem_st16(ta, v);
+              }
+            umma::fence_before_sync();
+            __syncthreads();
+          }
+          if (warp == 0) {  // O^T += V^T P^T over the round's pages (16 tokens each)
+            umma::fence_after_sync();
+            const int pr = min(kMpRound, np - r * kMpRound);
+            const uint32_t ka = kt_a + (r & 1) * kMpKtBytes, pa = pb_a + (r & 1) * (G * 128);
+#pragma unroll
+            for (int i = 0; i < DV / 128; ++i)
+#pragma unroll
+              for (int ks = 0; ks < kMpRound; ++ks)
+                if (ks < pr)
+                  umma::mma_bf16(tm + (uint32_t)(kMpOcol + G * i),
+                                 umma::sdesc_sw128(ka + 2 * i * (RT * 128) + ks * 2048, RT * 128, 1024),
+                                 umma::sdesc_sw128(pa + ks * 32, 16, 1024), kIdescO,
+                                 (r > 0 || ks > 0) ? 1u : 0u);
+            umma::commit(bars_a + 16);
+          }
         }
         cp_async_wait<0>();
-        // ---- finish: this lane holds heads g = 16 mt + lane/4 (+8), dims 64 warp + 8 nt + 2 (lane%4) (+1)
-        auto write_out = [&](float (&o)[G / 16][8][4], auto&& ml_of) {
+        if (nr > 0) {
+          bar_wait(2);
+          umma::fence_after_sync();
+        }
+        if (spart == 0) {
+          s_ml[2 * sh] = M_run;
+          s_ml[2 * sh + 1] = L_run;
+        }
+        // this thread's outputs: dims 128 (2 (w / 4) + bi) + 32 (w % 4) + lane, every head
+        const int sp = warp & 3, bh = warp >> 2;
+        float o[2][G];
+        if (nr > 0) {
 #pragma unroll
-          for (int mt = 0; mt < G / 16; ++mt)
+          for (int bi = 0; bi < 2; ++bi)
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const int g = mt * 16 + (lane >> 2) + 8 * hh;
-              const float2 ml = ml_of(g);
-              const float inv = ml.y > 0.0f ? 1.0f / ml.y : 0.0f;
+            for (int c = 0; c < G / 16; ++c) {
+              uint32_t v[16];
+              umma::tmem_ld16(tm + ((uint32_t)(32 * sp) << 16) +
+                                  (uint32_t)(kMpOcol + G * (2 * bh + bi) + 16 * c), v);
 #pragma unroll
-              for (int nt = 0; nt < 8; ++nt) {
-                const int d = warp * 64 + nt * 8 + 2 * (lane & 3);
-                __nv_bfloat162 v2;
-                v2.x = __float2bfloat16(o[mt][nt][2 * hh] * inv);
-                v2.y = __float2bfloat16(o[mt][nt][2 * hh + 1] * inv);
-                *reinterpret_cast<__nv_bfloat162*>(p.out + (orow + g) * DV + d) = v2;
-              }
-              if (warp == 0 && (lane & 3) == 0 && p.lse)
-                p.lse[orow + g] = ml.y > 0.0f ? (ml.x + log2f(ml.y)) * kLn2 : -INFINITY;
+              for (int j = 0; j < 16; ++j) o[bi][16 * c + j] = __uint_as_float(v[j]);
             }
+        } else {
+#pragma unroll
+          for (int bi = 0; bi < 2; ++bi)
+#pragma unroll
+            for (int h = 0; h < G; ++h) o[bi][h] = 0.0f;
+        }
+        umma::fence_before_sync();
+        __syncthreads();  // s_ml is complete
+        auto dim_of = [&](int bi) { return 128 * (2 * bh + bi) + 32 * sp + lane; };
+        // Results leave through shared memory (the K buffers are free now) and one bulk copy:
+        // the output rows of this request ([G][DV] bf16, contiguous), or a piece's partial
+        // ([G][DV + 2] fp32: unnormalised O, reference maximum, sum).
+        constexpr int PR = DV + 2;
+        constexpr uint32_t kPartBytes = G * PR * 4;
+        float* tile = reinterpret_cast<float*>(region);
+        const uint32_t tile_a = smem_u32(region);
+        auto store_out = [&](auto&& scale_of) {  // scale_of(h): the head's 1 / L
+          __nv_bfloat16* dst = p.out + orow * DV;
+          if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+            __nv_bfloat16* ot = reinterpret_cast<__nv_bfloat16*>(region);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float inv = scale_of(h);
+#pragma unroll
+              for (int bi = 0; bi < 2; ++bi) ot[h * DV + dim_of(bi)] = __float2bfloat16(o[bi][h] * inv);
+            }
+            umma::fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {  // the item's closing barrier waits for thread 0, so for the read
+              umma::bulk_s2g(dst, tile_a, G * DV * 2);
+              umma::bulk_wait_read();
+            }
+          } else {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float inv = scale_of(h);
+#pragma unroll
+              for (int bi = 0; bi < 2; ++bi) dst[h * DV + dim_of(bi)] = __float2bfloat16(o[bi][h] * inv);
+            }
+          }
         };
         if (Ab == 1) {
-          write_out(oacc, [&](int g) { return make_float2(s_ml[2 * g], s_ml[2 * g + 1]); });
+          store_out([&](int h) { return s_ml[2 * h + 1] > 0.0f ? 1.0f / s_ml[2 * h + 1] : 0.0f; });
+          if (spart == 0 && p.lse)
+            p.lse[orow + sh] = L_run > 0.0f ? (M_run + log2f(L_run)) * kLn2 : -INFINITY;
           if (tid == 0 && nch > 0) w.unit_done[b] = 0;
         } else if (piece < Ab - 1) {
           // publish this piece's partial and move on: the request's last piece merges them
-          float* dst = w.part + ((int64_t)b * A + piece) * G * (DV + 2);
 #pragma unroll
-          for (int mt = 0; mt < G / 16; ++mt)
+          for (int h = 0; h < G; ++h)
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const int g = mt * 16 + (lane >> 2) + 8 * hh;
-#pragma unroll
-              for (int nt = 0; nt < 8; ++nt) {
-                const int d = warp * 64 + nt * 8 + 2 * (lane & 3);
-                *reinterpret_cast<float2*>(dst + g * (DV + 2) + d) =
-                    make_float2(oacc[mt][nt][2 * hh], oacc[mt][nt][2 * hh + 1]);
-              }
-            }
-          for (int g = tid; g < G; g += NT)
-            *reinterpret_cast<float2*>(dst + g * (DV + 2) + DV) = make_float2(s_ml[2 * g], s_ml[2 * g + 1]);
+            for (int bi = 0; bi < 2; ++bi) tile[h * PR + dim_of(bi)] = o[bi][h];
+          if (spart == 0) {
+            tile[sh * PR + DV] = M_run;
+            tile[sh * PR + DV + 1] = L_run;
+          }
+          umma::fence_async_smem();
+          __syncthreads();
+          if (tid == 0) {  // complete before the count that publishes it (after the item)
+            umma::bulk_s2g(w.part + ((int64_t)b * A + piece) * G * PR, tile_a, kPartBytes);
+            umma::bulk_wait_done();
+          }
           pending = w.att_cnt + b;
         } else {
           // the last piece: wait for the other Ab - 1 partials (claimed before this item, and
-          // they never wait on a later one), then merge them into this piece's registers
+          // they never wait on a later one), then fold them in one at a time: each lands in
+          // shared memory with one bulk copy, and the running maximum and sum move with it
           if (tid == 0) s_misc[1] = mp_wait_at_least(w.att_cnt + b, Ab - 1, p.status) ? 1 : 0;
+          float* s_mm = reinterpret_cast<float*>(region + Ls.mm);  // [G][4]
+          for (int g = tid; g < G; g += NT) {
+            s_mm[4 * g] = s_ml[2 * g];
+            s_mm[4 * g + 1] = s_ml[2 * g + 1];
+          }
           __syncthreads();
           if (s_misc[1]) {
-            const float* src = w.part + (int64_t)b * A * G * (DV + 2);
-            // per head: the merged max and the rescaled sum (the page-max table is free again)
-            float* s_mm = s_pmax;  // [G][2]
-            for (int g = tid; g < G; g += NT) {
-              float M = s_ml[2 * g];
-              for (int q = 0; q < Ab - 1; ++q) M = fmaxf(M, __ldcg(src + (q * G + g) * (DV + 2) + DV));
-              float Lsum = (s_ml[2 * g] == -INFINITY) ? 0.0f : s_ml[2 * g + 1] * exp2f(s_ml[2 * g] - M);
-              for (int q = 0; q < Ab - 1; ++q) {
-                const float mq = __ldcg(src + (q * G + g) * (DV + 2) + DV);
-                if (mq != -INFINITY) Lsum = fmaf(__ldcg(src + (q * G + g) * (DV + 2) + DV + 1), exp2f(mq - M), Lsum);
+            const float* src = w.part + (int64_t)b * A * G * PR;
+            for (int q = 0; q < Ab - 1; ++q) {
+              if (tid == 0) {
+                umma::fence_async_global();
+                umma::mbar_expect_tx(bars_a + 24, kPartBytes);
+                umma::bulk_g2s(tile_a, src + (int64_t)q * G * PR, kPartBytes, bars_a + 24);
               }
-              s_mm[2 * g] = M;
-              s_mm[2 * g + 1] = Lsum;
+              bar_wait(3);
+              for (int g = tid; g < G; g += NT) {
+                const float mq = tile[g * PR + DV], lq = tile[g * PR + DV + 1];
+                const float M = s_mm[4 * g], Mn = fmaxf(M, mq);
+                const float fo = M == -INFINITY ? 0.0f : exp2f(M - Mn);
+                const float fq = mq == -INFINITY ? 0.0f : exp2f(mq - Mn);
+                s_mm[4 * g] = Mn;
+                s_mm[4 * g + 1] = fmaf(s_mm[4 * g + 1], fo, lq * fq);
+                s_mm[4 * g + 2] = fo;
+                s_mm[4 * g + 3] = fq;
+              }
+              __syncthreads();
+#pragma unroll
+              for (int h = 0; h < G; ++h) {
+                const float fo = s_mm[4 * h + 2], fq = s_mm[4 * h + 3];
+#pragma unroll
+                for (int bi = 0; bi < 2; ++bi)
+                  o[bi][h] = fmaf(tile[h * PR + dim_of(bi)], fq, o[bi][h] * fo);
+              }
+              __syncthreads();  // the tile is free for the next partial (or the output)
+            }
+            for (int g = tid; g < G; g += NT) {
+              const float M = s_mm[4 * g], Lsum = s_mm[4 * g + 1];
+              s_mm[4 * g + 2] = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
+              if (p.lse) p.lse[orow + g] = Lsum > 0.0f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
             }
             __syncthreads();
-#pragma unroll
-            for (int mt = 0; mt < G / 16; ++mt)
-#pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
-                const int g = mt * 16 + (lane >> 2) + 8 * hh;
-                const float M = s_mm[2 * g];
-                const float fo = (s_ml[2 * g] == -INFINITY) ? 0.0f : exp2f(s_ml[2 * g] - M);
-#pragma unroll
-                for (int nt = 0; nt < 8; ++nt) {
-                  oacc[mt][nt][2 * hh] *= fo;
-                  oacc[mt][nt][2 * hh + 1] *= fo;
-                }
-                for (int q = 0; q < Ab - 1; ++q) {
-                  const float* pq = src + (q * G + g) * (DV + 2);
-                  const float mq = __ldcg(pq + DV);
-                  const float f = (mq == -INFINITY) ? 0.0f : exp2f(mq - M);
-#pragma unroll
-                  for (int nt = 0; nt < 8; ++nt) {
-                    const int d = warp * 64 + nt * 8 + 2 * (lane & 3);
-                    const float2 v = __ldcg(reinterpret_cast<const float2*>(pq + d));
-                    oacc[mt][nt][2 * hh] = fmaf(v.x, f, oacc[mt][nt][2 * hh]);
-                    oacc[mt][nt][2 * hh + 1] = fmaf(v.y, f, oacc[mt][nt][2 * hh + 1]);
-                  }
-                }
-              }
-            write_out(oacc, [&](int g) { return make_float2(s_mm[2 * g], s_mm[2 * g + 1]); });
+            store_out([&](int h) { return s_mm[4 * h + 2]; });
             if (tid == 0) {  // every piece is past its waits: reset the request's counters
               w.att_cnt[b] = 0;
               w.unit_done[b] = 0;
@@ -914,6 +997,13 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
       atomicAdd(pending, 1);
       pending = nullptr;
     }
+  }
+  // every MMA of this launch has completed (each attention item waits for its last one)
+  umma::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    umma::fence_after_sync();
+    umma::tmem_dealloc(tm, kMpTmemCols);
   }
 }
 
