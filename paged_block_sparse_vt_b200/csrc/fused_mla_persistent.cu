@@ -96,7 +96,7 @@ struct MpWs {
   uint32_t* ckey;      // [B][nch_max][kc]: ordered score keys of each chunk's top-k
   uint16_t* coff;      // [B][nch_max][kc]: their offsets in the chunk, ascending
   int32_t* cpid;       // [B][nch_max][kc]: their page ids (-1 where out of range)
-  float* part;         // [B][A][G][Dv+2]: attention partials (acc, max, sum; base-2 max)
+  float* part;         // [B][A][G][Dv+4]: attention partials (acc; base-2 max, sums, pad)
   MpGeom g;
 };
 
@@ -119,7 +119,7 @@ static MpWsLayout mp_ws_layout(const DecodeParams& p, int G, int64_t unit_cap) {
   L.ckey = o;      o += mp_align256(cand * sizeof(uint32_t));
   L.coff = o;      o += mp_align256(cand * sizeof(uint16_t));
   L.cpid = o;      o += mp_align256(cand * sizeof(int32_t));
-  L.part = o;      o += mp_align256(U * g.A * G * (kMpDv + 2) * sizeof(float));
+  L.part = o;      o += mp_align256(U * g.A * G * (kMpDv + 4) * sizeof(float));
   L.total = o;
   return L;
 }
@@ -141,7 +141,7 @@ __host__ __device__ inline MpSmem mp_smem_layout(int G, int B, const MpGeom& g) 
   s.qm = o;     o += align16(kMpD * 4);
   s.sel = o;    o += align16(kMpSelCap * 4);
   s.phys = o;   o += align16(kMpSelCap * 4);
-  s.ml = o;     o += align16(G * 2 * 4);
+  s.ml = o;     o += align16(G * 4 * 4);
   s.misc = o;   o += align16(64 * 4);
   s.tc = o;     o += 64;  // three mbarriers, the tensor-memory address
   o = (o + 1023) & ~1023;
@@ -163,7 +163,7 @@ __host__ __device__ inline MpSmem mp_smem_layout(int G, int B, const MpGeom& g) 
   s.pb = a; a += 2 * G * 128;
   s.sc = a; a += G * RT * 4;
   s.fac = a; a += align16(G * 4);
-  s.mm = a; a += align16(G * 4 * 4);
+  s.mm = a; a += align16(G * 8 * 4);
   int r = scan;
   if (merge > r) r = merge;
   if (a > r) r = a;
@@ -729,7 +729,11 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
         constexpr int TPH = NT / G;   // softmax threads per head
         constexpr int TPT = RT / TPH; // tokens per softmax thread
         const int sh = tid / TPH, spart = tid % TPH;  // this thread's head and token group
-        float M_run = -INFINITY, L_run = 0.0f;        // the head's reference maximum and sum
+        // the head's reference maximum, the sum of its bf16 weights (as the MMA reads them: O's
+        // normaliser) and the sum of the same weights unrounded (for the lse: with a reference
+        // below the maximum, the largest weight is not a power of two and its rounding would
+        // reach the lse)
+        float M_run = -INFINITY, L_run = 0.0f, Le_run = 0.0f;
         stage_round(0);
         stage_round(1);
         for (int r = 0; r < nr; ++r) {
@@ -787,18 +791,24 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
             for (int o = 1; o < TPH; o <<= 1) mr = fmaxf(mr, __shfl_xor_sync(kFull, mr, o));
             const float Mn = mr > M_run + kLazyRescale ? mr : M_run;
             const float fac = Mn == M_run ? 1.0f : (M_run == -INFINITY ? 0.0f : exp2f(M_run - Mn));
-            float ls = 0.0f;
+            float ls = 0.0f, le = 0.0f;
             uint32_t pk[TPT / 2];
 #pragma unroll
             for (int i = 0; i < TPT; i += 2) {
-              const __nv_bfloat16 p0 = __float2bfloat16(sv[i] == -INFINITY ? 0.0f : exp2f(sv[i] - Mn));
-              const __nv_bfloat16 p1 = __float2bfloat16(sv[i + 1] == -INFINITY ? 0.0f : exp2f(sv[i + 1] - Mn));
+              const float e0 = sv[i] == -INFINITY ? 0.0f : exp2f(sv[i] - Mn);
+              const float e1 = sv[i + 1] == -INFINITY ? 0.0f : exp2f(sv[i + 1] - Mn);
+              const __nv_bfloat16 p0 = __float2bfloat16(e0), p1 = __float2bfloat16(e1);
               ls += __bfloat162float(p0) + __bfloat162float(p1);  // the weights the MMA reads
+              le += e0 + e1;
               pk[i / 2] = (uint32_t)__bfloat16_as_ushort(p0) | ((uint32_t)__bfloat16_as_ushort(p1) << 16);
             }
 #pragma unroll
-            for (int o = 1; o < TPH; o <<= 1) ls += __shfl_xor_sync(kFull, ls, o);
+            for (int o = 1; o < TPH; o <<= 1) {
+              ls += __shfl_xor_sync(kFull, ls, o);
+              le += __shfl_xor_sync(kFull, le, o);
+            }
             L_run = fmaf(L_run, fac, ls);
+            Le_run = fmaf(Le_run, fac, le);
             M_run = Mn;
             unsigned char* prow = region + Ls.pb + (r & 1) * (G * 128);
             if constexpr (TPT == 8) {
@@ -854,8 +864,9 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
           umma::fence_after_sync();
         }
         if (spart == 0) {
-          s_ml[2 * sh] = M_run;
-          s_ml[2 * sh + 1] = L_run;
+          s_ml[4 * sh] = M_run;
+          s_ml[4 * sh + 1] = L_run;
+          s_ml[4 * sh + 2] = Le_run;
         }
         // this thread's outputs: dims 128 (2 (w / 4) + bi) + 32 (w % 4) + lane, every head
         const int sp = warp & 3, bh = warp >> 2;
@@ -882,8 +893,8 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
         auto dim_of = [&](int bi) { return 128 * (2 * bh + bi) + 32 * sp + lane; };
         // Results leave through shared memory (the K buffers are free now) and one bulk copy:
         // the output rows of this request ([G][DV] bf16, contiguous), or a piece's partial
-        // ([G][DV + 2] fp32: unnormalised O, reference maximum, sum).
-        constexpr int PR = DV + 2;
+        // ([G][DV + 4] fp32: unnormalised O, reference maximum, the two sums, pad).
+        constexpr int PR = DV + 4;
         constexpr uint32_t kPartBytes = G * PR * 4;
         float* tile = reinterpret_cast<float*>(region);
         const uint32_t tile_a = smem_u32(region);
@@ -913,9 +924,9 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
           }
         };
         if (Ab == 1) {
-          store_out([&](int h) { return s_ml[2 * h + 1] > 0.0f ? 1.0f / s_ml[2 * h + 1] : 0.0f; });
+          store_out([&](int h) { return s_ml[4 * h + 1] > 0.0f ? 1.0f / s_ml[4 * h + 1] : 0.0f; });
           if (spart == 0 && p.lse)
-            p.lse[orow + sh] = L_run > 0.0f ? (M_run + log2f(L_run)) * kLn2 : -INFINITY;
+            p.lse[orow + sh] = Le_run > 0.0f ? (M_run + log2f(Le_run)) * kLn2 : -INFINITY;
           if (tid == 0 && nch > 0) w.unit_done[b] = 0;
         } else if (piece < Ab - 1) {
           // publish this piece's partial and move on: the request's last piece merges them
@@ -926,6 +937,8 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
           if (spart == 0) {
             tile[sh * PR + DV] = M_run;
             tile[sh * PR + DV + 1] = L_run;
+            tile[sh * PR + DV + 2] = Le_run;
+            tile[sh * PR + DV + 3] = 0.0f;
           }
           umma::fence_async_smem();
           __syncthreads();
@@ -939,10 +952,12 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
           // they never wait on a later one), then fold them in one at a time: each lands in
           // shared memory with one bulk copy, and the running maximum and sum move with it
           if (tid == 0) s_misc[1] = mp_wait_at_least(w.att_cnt + b, Ab - 1, p.status) ? 1 : 0;
-          float* s_mm = reinterpret_cast<float*>(region + Ls.mm);  // [G][4]
+          // per head: [0] maximum, [1] [2] the two sums, [3] [4] the factors of this step, [5] 1/L
+          float* s_mm = reinterpret_cast<float*>(region + Ls.mm);  // [G][8]
           for (int g = tid; g < G; g += NT) {
-            s_mm[4 * g] = s_ml[2 * g];
-            s_mm[4 * g + 1] = s_ml[2 * g + 1];
+            s_mm[8 * g] = s_ml[4 * g];
+            s_mm[8 * g + 1] = s_ml[4 * g + 1];
+            s_mm[8 * g + 2] = s_ml[4 * g + 2];
           }
           __syncthreads();
           if (s_misc[1]) {
@@ -955,19 +970,20 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
               }
               bar_wait(3);
               for (int g = tid; g < G; g += NT) {
-                const float mq = tile[g * PR + DV], lq = tile[g * PR + DV + 1];
-                const float M = s_mm[4 * g], Mn = fmaxf(M, mq);
+                const float mq = tile[g * PR + DV];
+                const float M = s_mm[8 * g], Mn = fmaxf(M, mq);
                 const float fo = M == -INFINITY ? 0.0f : exp2f(M - Mn);
                 const float fq = mq == -INFINITY ? 0.0f : exp2f(mq - Mn);
-                s_mm[4 * g] = Mn;
-                s_mm[4 * g + 1] = fmaf(s_mm[4 * g + 1], fo, lq * fq);
-                s_mm[4 * g + 2] = fo;
-                s_mm[4 * g + 3] = fq;
+                s_mm[8 * g] = Mn;
+                s_mm[8 * g + 1] = fmaf(s_mm[8 * g + 1], fo, tile[g * PR + DV + 1] * fq);
+                s_mm[8 * g + 2] = fmaf(s_mm[8 * g + 2], fo, tile[g * PR + DV + 2] * fq);
+                s_mm[8 * g + 3] = fo;
+                s_mm[8 * g + 4] = fq;
               }
               __syncthreads();
 #pragma unroll
               for (int h = 0; h < G; ++h) {
-                const float fo = s_mm[4 * h + 2], fq = s_mm[4 * h + 3];
+                const float fo = s_mm[8 * h + 3], fq = s_mm[8 * h + 4];
 #pragma unroll
                 for (int bi = 0; bi < 2; ++bi)
                   o[bi][h] = fmaf(tile[h * PR + dim_of(bi)], fq, o[bi][h] * fo);
@@ -975,12 +991,12 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
               __syncthreads();  // the tile is free for the next partial (or the output)
             }
             for (int g = tid; g < G; g += NT) {
-              const float M = s_mm[4 * g], Lsum = s_mm[4 * g + 1];
-              s_mm[4 * g + 2] = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
-              if (p.lse) p.lse[orow + g] = Lsum > 0.0f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+              const float M = s_mm[8 * g], Lsum = s_mm[8 * g + 1], Le = s_mm[8 * g + 2];
+              s_mm[8 * g + 5] = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
+              if (p.lse) p.lse[orow + g] = Le > 0.0f ? (M + log2f(Le)) * kLn2 : -INFINITY;
             }
             __syncthreads();
-            store_out([&](int h) { return s_mm[4 * h + 2]; });
+            store_out([&](int h) { return s_mm[8 * h + 5]; });
             if (tid == 0) {  // every piece is past its waits: reset the request's counters
               w.att_cnt[b] = 0;
               w.unit_done[b] = 0;
