@@ -128,7 +128,7 @@ static MpWsLayout mp_ws_layout(const DecodeParams& p, int G, int64_t unit_cap) {
 
 struct MpSmem {
   int prefix, keys, pids, qm, sel, phys, ml, misc, tc, region;  // region: one phase at a time
-  int ring, q, kt, pb, sc, fac, mm;                             // region offsets
+  int q, kt, pb, sc, fac, mm;                                   // region offsets (attention)
   int total;  // including 1 KB to align the base to the 1024-byte swizzle atoms
 };
 
@@ -143,11 +143,11 @@ __host__ __device__ inline MpSmem mp_smem_layout(int G, int B, const MpGeom& g) 
   s.phys = o;   o += align16(kMpSelCap * 4);
   s.ml = o;     o += align16(G * 4 * 4);
   s.misc = o;   o += align16(64 * 4);
-  s.tc = o;     o += 64;  // three mbarriers, the tensor-memory address
+  s.tc = o;     o += 64;  // four mbarriers, the tensor-memory address
   o = (o + 1023) & ~1023;
   s.region = o;
-  // scan: per-warp rings of centroid rows (the chunk top-k scratch reuses warp 0's ring)
-  s.ring = 0;
+  // scan: per-warp rings of centroid rows from offset 0 (the chunk top-k scratch reuses warp
+  // 0's ring)
   const int scan = kMpWarps * kMpScanSlots * kMpScanRows * kMpD * 4;
   // merge of the request's candidates: keys, logical pages, page ids, top-k scratch
   const int merge_small = 3 * 2 * kMpThreads * 4 + SmallTopk<kMpThreads>::BYTES;
