@@ -570,6 +570,27 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
         cp_async_commit();
       };
       if (q_early) stage_q();
+      auto phys_of = [&](int lp) {
+        int pg = ptrow[lp];
+        if (pg < 0 || pg >= p.num_pages) {
+          flag(p.status, VT_DEV_BAD_PAGE);
+          pg = -1;
+        }
+        return pg;
+      };
+      if (nch > 0) {
+        // the piece's reserved pages need no score: warp 1 loads their page ids while thread 0
+        // waits for the request's chunks below
+        const int bos = p.bos, topk = p.topk;
+        for (int q = tid - 32; q < np; q += NT) {
+          const int pos = j0 + q;
+          if (q >= 0 && (pos < bos || pos >= bos + topk)) {
+            const int lp = pos < bos ? pos : n - p.eos + (pos - bos - topk);
+            s_sel[q] = lp;
+            s_phys[q] = phys_of(lp);
+          }
+        }
+      }
       int ok = 1;
       if (nch > 0) {  // every chunk of the request has stored its candidates
         if (tid == 0) s_misc[1] = mp_wait_at_least(w.unit_done + b, nch, p.status) ? 1 : 0;
@@ -578,29 +599,13 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
       }
       if (ok) {
         // ---- the logical pages of this piece into s_sel[0, np), their page ids into s_phys
-        auto phys_of = [&](int lp) {
-          int pg = ptrow[lp];
-          if (pg < 0 || pg >= p.num_pages) {
-            flag(p.status, VT_DEV_BAD_PAGE);
-            pg = -1;
-          }
-          return pg;
-        };
         bool have_phys = false;
         if (nch > 0) {
           const int m = n - p.bos - p.eos;
           const int kc = gm.kc;
           const int C = (nch - 1) * kc + min(kc, m - (nch - 1) * kMlaChunk);
           const int64_t cb = (int64_t)b * gm.nch_max * kc;  // chunks are contiguous
-          const int bos = p.bos, topk = p.topk;
-          for (int q = tid; q < np; q += NT) {  // reserved pages of the piece
-            const int pos = j0 + q;
-            if (pos < bos || pos >= bos + topk) {
-              const int lp = pos < bos ? pos : n - p.eos + (pos - bos - topk);
-              s_sel[q] = lp;
-              s_phys[q] = phys_of(lp);
-            }
-          }
+          const int bos = p.bos, topk = p.topk;  // (the reserved pages are in s_sel already)
           if (write_sel) {
             for (int j = tid; j < bos; j += NT) selrow[j] = j;
             for (int j = tid; j < p.eos; j += NT) selrow[bos + topk + j] = n - p.eos + j;
