@@ -19,8 +19,9 @@
 //                   fp32 mean of the unit's G query heads; the CTA then takes the exact top-k
 //                   of the chunk in shared memory and stores those candidates (ordered
 //                   score key and offset, ascending by page) before counting the chunk done.
-//                   When the next item is a scan item too, its page ids and first batches
-//                   are put in flight before that top-k, so the CTA's loads do not pause.
+//                   When the next item is a scan item too, its page ids and query rows load
+//                   while that top-k runs, and its first batches go out right after it
+//                   (issuing them before the top-k measured slower).
 //                   The union of the chunks' top-k holds the unit's top-k: a key outside its
 //                   chunk's top-k has k keys above it in that chunk alone;
 //   attention    -- (unit, piece of at most kPiecePages selected pages), after every scan item.  The
