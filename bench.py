@@ -735,13 +735,18 @@ def measure_config(vt, cfg: int, dev, peak: float, iters: int = 10) -> dict:
                                            vb["select"])
         res["select_only_lossy"] = row(graph_time_ms([select_lossy(d) for d in ds], iters, dev),
                                        vb["select"])
-    if cfg in (2, 3):
+    if cfg == 4:  # the MLA split calls: the cluster kernel, and the persistent kernel's modes
+        res["select_only"] = row(graph_time_ms([select(d) for d in ds], iters, dev), vb["select"])
+        res["select_only_workspace"] = row(graph_time_ms([select_ws(d) for d in ds], iters, dev),
+                                           vb["select"])
+    if cfg in (2, 3, 4):
         for d in ds:
             select(d)()
         res["decode_only"] = row(graph_time_ms([decode(d) for d in ds], iters, dev), vb["decode"])
         res["select_then_decode"] = row(
             graph_time_ms([(lambda d=d: (select(d)(), decode(d)())) for d in ds], iters, dev),
             vb["select"] + vb["decode"])
+    if cfg in (2, 3, 4):
         for d in ds:
             d["ws_dec"] = vt.decode_workspace(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
                                               d["seq_lens"], d["sel"], head_dim_v=c.Dv)

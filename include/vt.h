@@ -143,11 +143,12 @@ vt_status vt_select_pages(const vt_paged_kv* kv, const vt_decode_args* a, int32_
 
 /*
  * vt_select_pages with a workspace (vt_fused_workspace_size() bytes, 256-byte aligned, zeroed
- * once, shared with the fused call under the same rules): for GQA heads and B <= 2048 the
- * selection then runs on the fused call's persistent CTAs, scan items only, the unit's last
- * counted chunk merging its candidates ("a workload planner for balanced GPU scheduling",
- * rndamp.com article, "A dual-stage programmable abstraction").  Same results and errors as
- * vt_select_pages; without a workspace, or for the MLA form, it is vt_select_pages.
+ * once, shared with the fused call under the same rules): for B <= 2048 the selection then
+ * runs on the fused call's persistent CTAs (GQA heads: scan items only, the unit's last
+ * counted chunk merging its candidates; the MLA form: scan items and one merge item per
+ * request) ("a workload planner for balanced GPU scheduling", rndamp.com article, "A
+ * dual-stage programmable abstraction").  Same results and errors as vt_select_pages;
+ * without a workspace, or for B > 2048, it is vt_select_pages.
  */
 vt_status vt_select_pages_ws(const vt_paged_kv* kv, const vt_decode_args* a, int32_t* sel,
                              int32_t* n_sel, void* workspace, size_t workspace_bytes,
@@ -185,10 +186,10 @@ vt_status vt_sparse_decode(const vt_paged_kv* kv, const vt_decode_args* a, const
                            const int32_t* n_sel, void* out, float* lse, void* stream);
 
 /*
- * vt_sparse_decode with a workspace (as for vt_select_pages_ws): for GQA heads and B <= 2048
- * the attention then runs on the fused call's persistent CTAs, attention items only, reading
- * the given selection.  Same results and errors as vt_sparse_decode; without a workspace, or
- * for the MLA form, it is vt_sparse_decode.
+ * vt_sparse_decode with a workspace (as for vt_select_pages_ws): for B <= 2048 (GQA heads and
+ * the MLA form) the attention then runs on the fused call's persistent CTAs, attention items
+ * only, reading the given selection.  Same results and errors as vt_sparse_decode; without a
+ * workspace, or for B > 2048, it is vt_sparse_decode.
  */
 vt_status vt_sparse_decode_ws(const vt_paged_kv* kv, const vt_decode_args* a, const int32_t* sel,
                               const int32_t* n_sel, void* out, float* lse, void* workspace,

@@ -190,7 +190,7 @@ def vt_select_pages(q, k_pool, v_pool, page_table, seq_lens, centroids, topk, bo
     """Top-k page selection per (request, KV head).  Returns (sel [B,Hkv,kmax], n_sel [B,Hkv]).
 
     With ``workspace`` (from fused_workspace() for the same arguments) it calls
-    vt_select_pages_ws (the persistent kernel for GQA heads, B <= 2048)."""
+    vt_select_pages_ws (the persistent kernel, B <= 2048)."""
     lib = load_library()
     kv = paged_kv(k_pool, v_pool, head_dim_v)
     a = decode_args(q, page_table, seq_lens, centroids, topk, bos, eos, 1.0, order, status)
@@ -238,7 +238,7 @@ def vt_sparse_decode(q, k_pool, v_pool, page_table, seq_lens, sel, n_sel, sm_sca
     """Attention over a given page selection.  Returns (out [B,Hq,Dv] bf16, lse [B,Hq] or None).
 
     With ``workspace`` (decode_workspace() for these arguments) it calls vt_sparse_decode_ws
-    (the persistent kernel for GQA heads, B <= 2048)."""
+    (the persistent kernel, B <= 2048)."""
     lib = load_library()
     kv = paged_kv(k_pool, v_pool, head_dim_v)
     kmax = sel.shape[2]

@@ -24,7 +24,7 @@ size_t mla_persist_workspace_bytes(const DecodeParams& p, int G, int64_t unit_ca
 int mla_persist_smem_bytes(const DecodeParams& p, int G);
 int mla_persist_max_batch();
 cudaError_t launch_mla_persist(const DecodeParams& p, int G, void* ws, int64_t unit_cap,
-                               int sm_count, cudaStream_t s);
+                               int sm_count, cudaStream_t s, int mode);
 cudaError_t launch_persist_fused(const DecodeParams& p, int D, int G, void* ws, int64_t unit_cap,
                                  int sm_count, cudaStream_t s, int mode);
 }  // namespace vt
@@ -241,9 +241,8 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
   p.n_fill = n_fill;
   p.cent_out = cent_out;
   // the select-only and decode-only calls given a workspace run as modes of the persistent
-  // GQA kernel (the MLA form keeps its cluster kernels for them)
-  const bool persistent = use_persistent(sh, a) &&
-                          (mode == kFused || (split_on_persistent && sh.path == kPathGqa && ws));
+  // kernels
+  const bool persistent = use_persistent(sh, a) && (mode == kFused || (split_on_persistent && ws));
   if (persistent) {
     const size_t need = persist_bytes(sh, p, unit_cap);
     if (!ws || ws_bytes < need)
@@ -255,7 +254,7 @@ vt_status launch_query_side(const vt_paged_kv* kv, const vt_decode_args* a, int 
                                           : persist_smem_bytes(p, sh.D, sh.G);
     if (bytes > 227 * 1024) return fail(VT_ERR_UNSUPPORTED, "shared memory need %d B too large", bytes);
     cudaError_t e = sh.path == kPathMla
-                        ? launch_mla_persist(p, sh.G, ws, unit_cap, sm_count(), st)
+                        ? launch_mla_persist(p, sh.G, ws, unit_cap, sm_count(), st, mode)
                         : launch_persist_fused(p, sh.D, sh.G, ws, unit_cap, sm_count(), st, mode);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return ok();

@@ -192,7 +192,9 @@ __device__ __forceinline__ bool mp_wait_at_least(const int32_t* ctr, int target,
   }
 }
 
-template <int G>
+// MODE: kFused, kSelect or kDecode (a template argument, so that the fused launch carries none
+// of the other modes' code)
+template <int G, int MODE>
 __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const DecodeParams p,
                                                                     const MpWs w) {
   constexpr int NT = kMpThreads;
@@ -283,7 +285,8 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
     const int i0 = min(p.B, tid * per), i1 = min(p.B, i0 + per);
     int run = 0;
     for (int i = i0; i < i1; ++i) {
-      const int c = mp_chunks(p.seq_lens[i], p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
+      const int c = MODE == kDecode ? 0
+                                      : mp_chunks(p.seq_lens[i], p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
       s_prefix[i] = c;
       run += c;
     }
@@ -315,7 +318,7 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
   // 17-page pieces and 256-page chunks 2 / 3 / 5 rounds gave 84.0 / 75.0 / 75.1 us).  Every
   // wait is still for items earlier in the queue.
   const int scan_items = s_prefix[p.B];
-  const int A = gm.A;
+  const int A = MODE == kSelect ? 1 : gm.A;  // items per request after its scans
   const int avg = (scan_items + p.B - 1) / p.B;
   const int lag = min(p.B, 5 * ((int)gridDim.x / (avg + A) + 1));  // ~5 rounds of CTAs
   const int total_items = scan_items + p.B * A;
@@ -537,29 +540,46 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
       pending = w.unit_done + b;
     } else {
       // ---------------------------------------------------------------- attention item
+      // (select-only calls: the request's merge item, which writes its selection and stops;
+      // decode-only calls: the selection is an input)
+      constexpr bool dec = MODE == kDecode, selm = MODE == kSelect;
       const int b = ib, piece = ic;
       const int Ab = A, ppb = gm.pp;
       const int L = p.seq_lens[b];
       const int n = (L + kPage - 1) / kPage;
       const bool valid = L >= 1 && n <= p.pt_stride;
       const bool dense = n <= p.kmax;
-      const int nch = mp_chunks(L, p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
-      const int ns = !valid ? 0 : (dense ? n : p.kmax);
+      const int nch = dec ? 0 : mp_chunks(L, p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
+      int ns = !valid ? 0 : (dense ? n : p.kmax);
+      if (dec) {
+        // every piece checks the request's whole row, so that a bad entry anywhere zeroes all
+        // of the request's outputs
+        const int nsi = valid ? p.n_sel[b] : 0;
+        int bad = valid && (nsi < 0 || nsi > p.kmax);
+        if (!bad)
+          for (int j = tid; j < nsi; j += NT) {
+            const int v = p.sel[(int64_t)b * p.kmax + j];
+            bad |= v < 0 || v >= n;
+          }
+        bad = __syncthreads_or(bad);
+        if (bad && tid == 0 && piece == 0) flag(p.status, VT_DEV_BAD_SEL);
+        ns = bad ? 0 : nsi;
+      }
       const int j0 = piece * ppb;
-      const int np = piece == Ab - 1 ? max(0, ns - j0) : max(0, min(ns - j0, ppb));
-      const bool write_sel = piece == 0 && p.sel != nullptr;
+      const int np = selm ? 0 : (piece == Ab - 1 ? max(0, ns - j0) : max(0, min(ns - j0, ppb)));
+      const bool write_sel = piece == 0 && p.sel != nullptr && !dec;
       int32_t* selrow = write_sel ? p.sel + (int64_t)b * p.kmax : nullptr;
       const int64_t orow = (int64_t)b * p.Hq;
       const int32_t* ptrow = p.page_table + (int64_t)b * p.pt_stride;
       if (tid == 0 && piece == 0) {
         if (!valid) flag(p.status, VT_DEV_BAD_LEN);
-        if (p.n_sel) p.n_sel[b] = ns;
+        if (p.n_sel && !dec) p.n_sel[b] = ns;
       }
       // Q (G x 576) for the attention below, fetched while the wait and the merge run (its slot
       // lies past every merge scratch of the small path)
       const int m_c = n - p.bos - p.eos;
       const int C_c = nch > 0 ? (nch - 1) * gm.kc + min(gm.kc, m_c - (nch - 1) * kMlaChunk) : 0;
-      const bool q_early = C_c <= 2 * NT;
+      const bool q_early = !selm && C_c <= 2 * NT;
       const uint32_t q_a = smem_u32(region + Ls.q);  // [atom][G rows][128 B], swizzled K-major
       auto stage_q = [&]() {
         for (int i = tid; i < G * (D / 8); i += NT) {
@@ -676,7 +696,8 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
           auto page_at = [&](int pos) {
             return (!resv || pos < p.bos) ? pos : n - p.eos + (pos - p.bos);
           };
-          for (int q = tid; q < np; q += NT) s_sel[q] = page_at(j0 + q);
+          for (int q = tid; q < np; q += NT)
+            s_sel[q] = dec ? p.sel[(int64_t)b * p.kmax + j0 + q] : page_at(j0 + q);
           if (write_sel)
             for (int j = tid; j < p.kmax; j += NT) selrow[j] = j < ns ? page_at(j) : -1;
         }
@@ -685,326 +706,331 @@ __global__ void __launch_bounds__(kMpThreads, 1) persist_mla_kernel(const Decode
           if (tid < np) s_phys[tid] = phys_of(s_sel[tid]);
           __syncthreads();
         }
-        // ---- the piece's pages in rounds of kMpRound pages (RT = 64 tokens) on the tensor cores.
-        // A round's K tile lands (zero rows past the valid tokens) in 128-byte swizzled K-major
-        // order in one of two buffers; per round
-        //   S^T = K Q^T      M = 64 tokens, N = G heads, K = 576, into tensor memory;
-        //   the softmax of each head against its reference maximum, through a shared-memory
-        //                    transpose of S^T (a group of NT / G threads per head); P in bf16,
-        //                    heads x tokens, as the next MMA's K-major operand;
-        //   O^T += V^T P^T   M = 128 output dims per block (four blocks), N = G, K = the round's
-        //                    tokens; V^T is the latent part of the same K tile, read MN-major;
-        //                    O^T stays in tensor memory for the whole piece.
-        // A head's reference maximum moves only when a round's maximum exceeds it by more than
-        // kLazyRescale (base 2), and O^T is then rescaled in tensor memory; P stays below 2^8.
-        // The tensor core runs round r's MMAs while round r + 1's tile lands in the other buffer.
-        unsigned char* kt = region + Ls.kt;
-        const uint32_t kt_a = smem_u32(kt), pb_a = smem_u32(region + Ls.pb);
-        float* s_sc = reinterpret_cast<float*>(region + Ls.sc);    // [G][RT] scores of the round
-        float* s_fac = reinterpret_cast<float*>(region + Ls.fac);  // [G] rescale factors
-        const int last_valid = L - kPage * (n - 1);
-        if (!q_early) stage_q();
-        const int nr = (np + kMpRound - 1) / kMpRound;
-        auto row_ok = [&](int j, int tt) {  // token tt of the piece's j-th page is attended
-          return j < np && s_phys[j] >= 0 && (s_sel[j] != n - 1 || tt < last_valid);
-        };
-        // staging: thread t copies rows t / 8 and t / 8 + 32 of the round, 16-byte chunk t % 8
-        // of each of the nine 128-byte atoms (eight threads read 128 contiguous bytes of a row)
-        static_assert(NT == 4 * RT, "eight threads per row, two rows per thread");
-        const int st_c = tid & 7;
-        auto stage_round = [&](int r) {  // every thread commits one group per call
-          if (r < nr) {
-            const uint32_t buf = kt_a + (r & 1) * kMpKtBytes;
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int row = (tid >> 3) + 32 * h2;
-              const int j = r * kMpRound + row / kPage, tt = row % kPage;
-              const bool ok_row = row_ok(j, tt);
-              const __nv_bfloat16* src =
-                  ok_row ? p.k_pool + (int64_t)s_phys[j] * p.sk_p + (int64_t)tt * p.sk_t + st_c * 8
-                         : p.k_pool;
-              const uint32_t dst = buf + umma::sw128_off(row, st_c);
-#pragma unroll
-              for (int kb = 0; kb < D / 64; ++kb)
-                cp_async16(dst + kb * (RT * 128), src + (ok_row ? kb * 64 : 0), ok_row ? 16 : 0);
-            }
-          }
-          cp_async_commit();
-        };
-        constexpr int TPH = NT / G;   // softmax threads per head
-        constexpr int TPT = RT / TPH; // tokens per softmax thread
-        const int sh = tid / TPH, spart = tid % TPH;  // this thread's head and token group
-        // the head's reference maximum, the sum of its bf16 weights (as the MMA reads them: O's
-        // normaliser) and the sum of the same weights unrounded (for the lse: with a reference
-        // below the maximum, the largest weight is not a power of two and its rounding would
-        // reach the lse)
-        float M_run = -INFINITY, L_run = 0.0f, Le_run = 0.0f;
-        stage_round(0);
-        stage_round(1);
-        for (int r = 0; r < nr; ++r) {
-          // round r has landed (and Q with it): S^T(r) on the tensor core
-          if (r == 0) cp_async_wait<1>(); else cp_async_wait<0>();
-          umma::fence_async_smem();
-          __syncthreads();
-          if (warp == 0) {
-            umma::fence_after_sync();
-            const uint32_t ka = kt_a + (r & 1) * kMpKtBytes;
-            const uint32_t d = tm + (uint32_t)((r & 1) * G);
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks)
-              umma::mma_bf16(d, umma::sdesc_sw128(ka + (ks >> 2) * (RT * 128) + (ks & 3) * 32, 16, 1024),
-                             umma::sdesc_sw128(q_a + (ks >> 2) * (G * 128) + (ks & 3) * 32, 16, 1024),
-                             kIdescS, ks > 0 ? 1u : 0u);
-            umma::commit(bars_a + 8 * (r & 1));
-          }
-          if (r >= 1) {
-            // O^T(r - 1) has completed (its commit is waited on once), so the buffer it read
-            // takes round r + 1
-            bar_wait(2);
-            if (r + 1 < nr) stage_round(r + 1);
-          }
-          bar_wait(r & 1);
-          umma::fence_after_sync();
-          if (warp < 4) {  // token 16 w + lane (lane < 16) sits in lane 32 w + lane
-            uint32_t v[G / 16][16];
-#pragma unroll
-            for (int c = 0; c < G / 16; ++c)
-              umma::tmem_ld16(tm + ((uint32_t)(32 * warp) << 16) + (uint32_t)((r & 1) * G + 16 * c), v[c]);
-            umma::fence_before_sync();
-            if (lane < 16) {
-              const bool ok = row_ok(r * kMpRound + warp, lane);
-              const int t = 16 * warp + lane;
-#pragma unroll
-              for (int h = 0; h < G; ++h)
-                s_sc[h * RT + t] = ok ? __uint_as_float(v[h >> 4][h & 15]) * p.qscale : -INFINITY;
-            }
-          }
-          __syncthreads();
-          // softmax of head sh over tokens [TPT spart, TPT spart + TPT) of the round
-          int need = 0;
-          {
-            float sv[TPT];
-#pragma unroll
-            for (int i = 0; i < TPT; i += 4) {
-              const float4 f4 = *reinterpret_cast<const float4*>(s_sc + sh * RT + spart * TPT + i);
-              sv[i] = f4.x; sv[i + 1] = f4.y; sv[i + 2] = f4.z; sv[i + 3] = f4.w;
-            }
-            float mr = sv[0];
-#pragma unroll
-            for (int i = 1; i < TPT; ++i) mr = fmaxf(mr, sv[i]);
-#pragma unroll
-            for (int o = 1; o < TPH; o <<= 1) mr = fmaxf(mr, __shfl_xor_sync(kFull, mr, o));
-            const float Mn = mr > M_run + kLazyRescale ? mr : M_run;
-            const float fac = Mn == M_run ? 1.0f : (M_run == -INFINITY ? 0.0f : exp2f(M_run - Mn));
-            float ls = 0.0f, le = 0.0f;
-            uint32_t pk[TPT / 2];
-#pragma unroll
-            for (int i = 0; i < TPT; i += 2) {
-              const float e0 = sv[i] == -INFINITY ? 0.0f : exp2f(sv[i] - Mn);
-              const float e1 = sv[i + 1] == -INFINITY ? 0.0f : exp2f(sv[i + 1] - Mn);
-              const __nv_bfloat16 p0 = __float2bfloat16(e0), p1 = __float2bfloat16(e1);
-              ls += __bfloat162float(p0) + __bfloat162float(p1);  // the weights the MMA reads
-              le += e0 + e1;
-              pk[i / 2] = (uint32_t)__bfloat16_as_ushort(p0) | ((uint32_t)__bfloat16_as_ushort(p1) << 16);
-            }
-#pragma unroll
-            for (int o = 1; o < TPH; o <<= 1) {
-              ls += __shfl_xor_sync(kFull, ls, o);
-              le += __shfl_xor_sync(kFull, le, o);
-            }
-            L_run = fmaf(L_run, fac, ls);
-            Le_run = fmaf(Le_run, fac, le);
-            M_run = Mn;
-            unsigned char* prow = region + Ls.pb + (r & 1) * (G * 128);
-            if constexpr (TPT == 8) {
-              *reinterpret_cast<uint4*>(prow + umma::sw128_off(sh, spart)) =
-                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            } else {
-              *reinterpret_cast<uint2*>(prow + umma::sw128_off(sh, spart >> 1) + (spart & 1) * 8) =
-                  make_uint2(pk[0], pk[1]);
-            }
-            if (spart == 0) s_fac[sh] = fac;
-            need = (r > 0 && fac != 1.0f) ? 1 : 0;
-          }
-          umma::fence_async_smem();  // P is read by the tensor core
-          if (__syncthreads_or(need)) {
-            // O^T *= fac per head (column); O^T(r - 1) has completed.  Warp w rescales blocks
-            // 2 (w / 4) and 2 (w / 4) + 1 in its lane quarter.
-            const int sp = warp & 3, bh = warp >> 2;
-#pragma unroll
-            for (int bi = 0; bi < 2; ++bi)
-#pragma unroll
-              for (int c = 0; c < G / 16; ++c) {
-                const uint32_t ta = tm + ((uint32_t)(32 * sp) << 16) +
-                                    (uint32_t)(kMpOcol + G * (2 * bh + bi) + 16 * c);
-                uint32_t v[16];
-                umma::tmem_ld16(ta, v);
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                  v[j] = __float_as_uint(__uint_as_float(v[j]) * s_fac[16 * c + j]);
-                umma::tmem_st16(ta, v);
-              }
-            umma::fence_before_sync();
-            __syncthreads();
-          }
-          if (warp == 0) {  // O^T += V^T P^T over the round's pages (16 tokens each)
-            umma::fence_after_sync();
-            const int pr = min(kMpRound, np - r * kMpRound);
-            const uint32_t ka = kt_a + (r & 1) * kMpKtBytes, pa = pb_a + (r & 1) * (G * 128);
-#pragma unroll
-            for (int i = 0; i < DV / 128; ++i)
-#pragma unroll
-              for (int ks = 0; ks < kMpRound; ++ks)
-                if (ks < pr)
-                  umma::mma_bf16(tm + (uint32_t)(kMpOcol + G * i),
-                                 umma::sdesc_sw128(ka + 2 * i * (RT * 128) + ks * 2048, RT * 128, 1024),
-                                 umma::sdesc_sw128(pa + ks * 32, 16, 1024), kIdescO,
-                                 (r > 0 || ks > 0) ? 1u : 0u);
-            umma::commit(bars_a + 16);
-          }
-        }
-        cp_async_wait<0>();
-        if (nr > 0) {
-          bar_wait(2);
-          umma::fence_after_sync();
-        }
-        if (spart == 0) {
-          s_ml[4 * sh] = M_run;
-          s_ml[4 * sh + 1] = L_run;
-          s_ml[4 * sh + 2] = Le_run;
-        }
-        // this thread's outputs: dims 128 (2 (w / 4) + bi) + 32 (w % 4) + lane, every head
-        const int sp = warp & 3, bh = warp >> 2;
-        float o[2][G];
-        if (nr > 0) {
-#pragma unroll
-          for (int bi = 0; bi < 2; ++bi)
-#pragma unroll
-            for (int c = 0; c < G / 16; ++c) {
-              uint32_t v[16];
-              umma::tmem_ld16(tm + ((uint32_t)(32 * sp) << 16) +
-                                  (uint32_t)(kMpOcol + G * (2 * bh + bi) + 16 * c), v);
-#pragma unroll
-              for (int j = 0; j < 16; ++j) o[bi][16 * c + j] = __uint_as_float(v[j]);
-            }
+        if (selm) {
+          // select-only: the request's selection is written; its chunk counter goes back to 0
+          if (tid == 0 && nch > 0) w.unit_done[b] = 0;
         } else {
-#pragma unroll
-          for (int bi = 0; bi < 2; ++bi)
-#pragma unroll
-            for (int h = 0; h < G; ++h) o[bi][h] = 0.0f;
-        }
-        umma::fence_before_sync();
-        __syncthreads();  // s_ml is complete
-        auto dim_of = [&](int bi) { return 128 * (2 * bh + bi) + 32 * sp + lane; };
-        // Results leave through shared memory (the K buffers are free now) and one bulk copy:
-        // the output rows of this request ([G][DV] bf16, contiguous), or a piece's partial
-        // ([G][DV + 4] fp32: unnormalised O, reference maximum, the two sums, pad).
-        constexpr int PR = DV + 4;
-        constexpr uint32_t kPartBytes = G * PR * 4;
-        float* tile = reinterpret_cast<float*>(region);
-        const uint32_t tile_a = smem_u32(region);
-        auto store_out = [&](auto&& scale_of) {  // scale_of(h): the head's 1 / L
-          __nv_bfloat16* dst = p.out + orow * DV;
-          if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
-            __nv_bfloat16* ot = reinterpret_cast<__nv_bfloat16*>(region);
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              const float inv = scale_of(h);
-#pragma unroll
-              for (int bi = 0; bi < 2; ++bi) ot[h * DV + dim_of(bi)] = __float2bfloat16(o[bi][h] * inv);
+          // ---- the piece's pages in rounds of kMpRound pages (RT = 64 tokens) on the tensor cores.
+          // A round's K tile lands (zero rows past the valid tokens) in 128-byte swizzled K-major
+          // order in one of two buffers; per round
+          //   S^T = K Q^T      M = 64 tokens, N = G heads, K = 576, into tensor memory;
+          //   the softmax of each head against its reference maximum, through a shared-memory
+          //                    transpose of S^T (a group of NT / G threads per head); P in bf16,
+          //                    heads x tokens, as the next MMA's K-major operand;
+          //   O^T += V^T P^T   M = 128 output dims per block (four blocks), N = G, K = the round's
+          //                    tokens; V^T is the latent part of the same K tile, read MN-major;
+          //                    O^T stays in tensor memory for the whole piece.
+          // A head's reference maximum moves only when a round's maximum exceeds it by more than
+          // kLazyRescale (base 2), and O^T is then rescaled in tensor memory; P stays below 2^8.
+          // The tensor core runs round r's MMAs while round r + 1's tile lands in the other buffer.
+          unsigned char* kt = region + Ls.kt;
+          const uint32_t kt_a = smem_u32(kt), pb_a = smem_u32(region + Ls.pb);
+          float* s_sc = reinterpret_cast<float*>(region + Ls.sc);    // [G][RT] scores of the round
+          float* s_fac = reinterpret_cast<float*>(region + Ls.fac);  // [G] rescale factors
+          const int last_valid = L - kPage * (n - 1);
+          if (!q_early) stage_q();
+          const int nr = (np + kMpRound - 1) / kMpRound;
+          auto row_ok = [&](int j, int tt) {  // token tt of the piece's j-th page is attended
+            return j < np && s_phys[j] >= 0 && (s_sel[j] != n - 1 || tt < last_valid);
+          };
+          // staging: thread t copies rows t / 8 and t / 8 + 32 of the round, 16-byte chunk t % 8
+          // of each of the nine 128-byte atoms (eight threads read 128 contiguous bytes of a row)
+          static_assert(NT == 4 * RT, "eight threads per row, two rows per thread");
+          const int st_c = tid & 7;
+          auto stage_round = [&](int r) {  // every thread commits one group per call
+            if (r < nr) {
+              const uint32_t buf = kt_a + (r & 1) * kMpKtBytes;
+  #pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const int row = (tid >> 3) + 32 * h2;
+                const int j = r * kMpRound + row / kPage, tt = row % kPage;
+                const bool ok_row = row_ok(j, tt);
+                const __nv_bfloat16* src =
+                    ok_row ? p.k_pool + (int64_t)s_phys[j] * p.sk_p + (int64_t)tt * p.sk_t + st_c * 8
+                           : p.k_pool;
+                const uint32_t dst = buf + umma::sw128_off(row, st_c);
+  #pragma unroll
+                for (int kb = 0; kb < D / 64; ++kb)
+                  cp_async16(dst + kb * (RT * 128), src + (ok_row ? kb * 64 : 0), ok_row ? 16 : 0);
+              }
+            }
+            cp_async_commit();
+          };
+          constexpr int TPH = NT / G;   // softmax threads per head
+          constexpr int TPT = RT / TPH; // tokens per softmax thread
+          const int sh = tid / TPH, spart = tid % TPH;  // this thread's head and token group
+          // the head's reference maximum, the sum of its bf16 weights (as the MMA reads them: O's
+          // normaliser) and the sum of the same weights unrounded (for the lse: with a reference
+          // below the maximum, the largest weight is not a power of two and its rounding would
+          // reach the lse)
+          float M_run = -INFINITY, L_run = 0.0f, Le_run = 0.0f;
+          stage_round(0);
+          stage_round(1);
+          for (int r = 0; r < nr; ++r) {
+            // round r has landed (and Q with it): S^T(r) on the tensor core
+            if (r == 0) cp_async_wait<1>(); else cp_async_wait<0>();
+            umma::fence_async_smem();
+            __syncthreads();
+            if (warp == 0) {
+              umma::fence_after_sync();
+              const uint32_t ka = kt_a + (r & 1) * kMpKtBytes;
+              const uint32_t d = tm + (uint32_t)((r & 1) * G);
+  #pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks)
+                umma::mma_bf16(d, umma::sdesc_sw128(ka + (ks >> 2) * (RT * 128) + (ks & 3) * 32, 16, 1024),
+                               umma::sdesc_sw128(q_a + (ks >> 2) * (G * 128) + (ks & 3) * 32, 16, 1024),
+                               kIdescS, ks > 0 ? 1u : 0u);
+              umma::commit(bars_a + 8 * (r & 1));
+            }
+            if (r >= 1) {
+              // O^T(r - 1) has completed (its commit is waited on once), so the buffer it read
+              // takes round r + 1
+              bar_wait(2);
+              if (r + 1 < nr) stage_round(r + 1);
+            }
+            bar_wait(r & 1);
+            umma::fence_after_sync();
+            if (warp < 4) {  // token 16 w + lane (lane < 16) sits in lane 32 w + lane
+              uint32_t v[G / 16][16];
+  #pragma unroll
+              for (int c = 0; c < G / 16; ++c)
+                umma::tmem_ld16(tm + ((uint32_t)(32 * warp) << 16) + (uint32_t)((r & 1) * G + 16 * c), v[c]);
+              umma::fence_before_sync();
+              if (lane < 16) {
+                const bool ok = row_ok(r * kMpRound + warp, lane);
+                const int t = 16 * warp + lane;
+  #pragma unroll
+                for (int h = 0; h < G; ++h)
+                  s_sc[h * RT + t] = ok ? __uint_as_float(v[h >> 4][h & 15]) * p.qscale : -INFINITY;
+              }
+            }
+            __syncthreads();
+            // softmax of head sh over tokens [TPT spart, TPT spart + TPT) of the round
+            int need = 0;
+            {
+              float sv[TPT];
+  #pragma unroll
+              for (int i = 0; i < TPT; i += 4) {
+                const float4 f4 = *reinterpret_cast<const float4*>(s_sc + sh * RT + spart * TPT + i);
+                sv[i] = f4.x; sv[i + 1] = f4.y; sv[i + 2] = f4.z; sv[i + 3] = f4.w;
+              }
+              float mr = sv[0];
+  #pragma unroll
+              for (int i = 1; i < TPT; ++i) mr = fmaxf(mr, sv[i]);
+  #pragma unroll
+              for (int o = 1; o < TPH; o <<= 1) mr = fmaxf(mr, __shfl_xor_sync(kFull, mr, o));
+              const float Mn = mr > M_run + kLazyRescale ? mr : M_run;
+              const float fac = Mn == M_run ? 1.0f : (M_run == -INFINITY ? 0.0f : exp2f(M_run - Mn));
+              float ls = 0.0f, le = 0.0f;
+              uint32_t pk[TPT / 2];
+  #pragma unroll
+              for (int i = 0; i < TPT; i += 2) {
+                const float e0 = sv[i] == -INFINITY ? 0.0f : exp2f(sv[i] - Mn);
+                const float e1 = sv[i + 1] == -INFINITY ? 0.0f : exp2f(sv[i + 1] - Mn);
+                const __nv_bfloat16 p0 = __float2bfloat16(e0), p1 = __float2bfloat16(e1);
+                ls += __bfloat162float(p0) + __bfloat162float(p1);  // the weights the MMA reads
+                le += e0 + e1;
+                pk[i / 2] = (uint32_t)__bfloat16_as_ushort(p0) | ((uint32_t)__bfloat16_as_ushort(p1) << 16);
+              }
+  #pragma unroll
+              for (int o = 1; o < TPH; o <<= 1) {
+                ls += __shfl_xor_sync(kFull, ls, o);
+                le += __shfl_xor_sync(kFull, le, o);
+              }
+              L_run = fmaf(L_run, fac, ls);
+              Le_run = fmaf(Le_run, fac, le);
+              M_run = Mn;
+              unsigned char* prow = region + Ls.pb + (r & 1) * (G * 128);
+              if constexpr (TPT == 8) {
+                *reinterpret_cast<uint4*>(prow + umma::sw128_off(sh, spart)) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              } else {
+                *reinterpret_cast<uint2*>(prow + umma::sw128_off(sh, spart >> 1) + (spart & 1) * 8) =
+                    make_uint2(pk[0], pk[1]);
+              }
+              if (spart == 0) s_fac[sh] = fac;
+              need = (r > 0 && fac != 1.0f) ? 1 : 0;
+            }
+            umma::fence_async_smem();  // P is read by the tensor core
+            if (__syncthreads_or(need)) {
+              // O^T *= fac per head (column); O^T(r - 1) has completed.  Warp w rescales blocks
+              // 2 (w / 4) and 2 (w / 4) + 1 in its lane quarter.
+              const int sp = warp & 3, bh = warp >> 2;
+  #pragma unroll
+              for (int bi = 0; bi < 2; ++bi)
+  #pragma unroll
+                for (int c = 0; c < G / 16; ++c) {
+                  const uint32_t ta = tm + ((uint32_t)(32 * sp) << 16) +
+                                      (uint32_t)(kMpOcol + G * (2 * bh + bi) + 16 * c);
+                  uint32_t v[16];
+                  umma::tmem_ld16(ta, v);
+  #pragma unroll
+                  for (int j = 0; j < 16; ++j)
+                    v[j] = __float_as_uint(__uint_as_float(v[j]) * s_fac[16 * c + j]);
+                  umma::tmem_st16(ta, v);
+                }
+              umma::fence_before_sync();
+              __syncthreads();
+            }
+            if (warp == 0) {  // O^T += V^T P^T over the round's pages (16 tokens each)
+              umma::fence_after_sync();
+              const int pr = min(kMpRound, np - r * kMpRound);
+              const uint32_t ka = kt_a + (r & 1) * kMpKtBytes, pa = pb_a + (r & 1) * (G * 128);
+  #pragma unroll
+              for (int i = 0; i < DV / 128; ++i)
+  #pragma unroll
+                for (int ks = 0; ks < kMpRound; ++ks)
+                  if (ks < pr)
+                    umma::mma_bf16(tm + (uint32_t)(kMpOcol + G * i),
+                                   umma::sdesc_sw128(ka + 2 * i * (RT * 128) + ks * 2048, RT * 128, 1024),
+                                   umma::sdesc_sw128(pa + ks * 32, 16, 1024), kIdescO,
+                                   (r > 0 || ks > 0) ? 1u : 0u);
+              umma::commit(bars_a + 16);
+            }
+          }
+          cp_async_wait<0>();
+          if (nr > 0) {
+            bar_wait(2);
+            umma::fence_after_sync();
+          }
+          if (spart == 0) {
+            s_ml[4 * sh] = M_run;
+            s_ml[4 * sh + 1] = L_run;
+            s_ml[4 * sh + 2] = Le_run;
+          }
+          // this thread's outputs: dims 128 (2 (w / 4) + bi) + 32 (w % 4) + lane, every head
+          const int sp = warp & 3, bh = warp >> 2;
+          float o[2][G];
+          if (nr > 0) {
+  #pragma unroll
+            for (int bi = 0; bi < 2; ++bi)
+  #pragma unroll
+              for (int c = 0; c < G / 16; ++c) {
+                uint32_t v[16];
+                umma::tmem_ld16(tm + ((uint32_t)(32 * sp) << 16) +
+                                    (uint32_t)(kMpOcol + G * (2 * bh + bi) + 16 * c), v);
+  #pragma unroll
+                for (int j = 0; j < 16; ++j) o[bi][16 * c + j] = __uint_as_float(v[j]);
+              }
+          } else {
+  #pragma unroll
+            for (int bi = 0; bi < 2; ++bi)
+  #pragma unroll
+              for (int h = 0; h < G; ++h) o[bi][h] = 0.0f;
+          }
+          umma::fence_before_sync();
+          __syncthreads();  // s_ml is complete
+          auto dim_of = [&](int bi) { return 128 * (2 * bh + bi) + 32 * sp + lane; };
+          // Results leave through shared memory (the K buffers are free now) and one bulk copy:
+          // the output rows of this request ([G][DV] bf16, contiguous), or a piece's partial
+          // ([G][DV + 4] fp32: unnormalised O, reference maximum, the two sums, pad).
+          constexpr int PR = DV + 4;
+          constexpr uint32_t kPartBytes = G * PR * 4;
+          float* tile = reinterpret_cast<float*>(region);
+          const uint32_t tile_a = smem_u32(region);
+          auto store_out = [&](auto&& scale_of) {  // scale_of(h): the head's 1 / L
+            __nv_bfloat16* dst = p.out + orow * DV;
+            if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+              __nv_bfloat16* ot = reinterpret_cast<__nv_bfloat16*>(region);
+  #pragma unroll
+              for (int h = 0; h < G; ++h) {
+                const float inv = scale_of(h);
+  #pragma unroll
+                for (int bi = 0; bi < 2; ++bi) ot[h * DV + dim_of(bi)] = __float2bfloat16(o[bi][h] * inv);
+              }
+              umma::fence_async_smem();
+              __syncthreads();
+              if (tid == 0) {  // the item's closing barrier waits for thread 0, so for the read
+                umma::bulk_s2g(dst, tile_a, G * DV * 2);
+                umma::bulk_wait_read();
+              }
+            } else {
+  #pragma unroll
+              for (int h = 0; h < G; ++h) {
+                const float inv = scale_of(h);
+  #pragma unroll
+                for (int bi = 0; bi < 2; ++bi) dst[h * DV + dim_of(bi)] = __float2bfloat16(o[bi][h] * inv);
+              }
+            }
+          };
+          if (Ab == 1) {
+            store_out([&](int h) { return s_ml[4 * h + 1] > 0.0f ? 1.0f / s_ml[4 * h + 1] : 0.0f; });
+            if (spart == 0 && p.lse)
+              p.lse[orow + sh] = Le_run > 0.0f ? (M_run + log2f(Le_run)) * kLn2 : -INFINITY;
+            if (tid == 0 && nch > 0) w.unit_done[b] = 0;
+          } else if (piece < Ab - 1) {
+            // publish this piece's partial and move on: the request's last piece merges them
+  #pragma unroll
+            for (int h = 0; h < G; ++h)
+  #pragma unroll
+              for (int bi = 0; bi < 2; ++bi) tile[h * PR + dim_of(bi)] = o[bi][h];
+            if (spart == 0) {
+              tile[sh * PR + DV] = M_run;
+              tile[sh * PR + DV + 1] = L_run;
+              tile[sh * PR + DV + 2] = Le_run;
+              tile[sh * PR + DV + 3] = 0.0f;
             }
             umma::fence_async_smem();
             __syncthreads();
-            if (tid == 0) {  // the item's closing barrier waits for thread 0, so for the read
-              umma::bulk_s2g(dst, tile_a, G * DV * 2);
-              umma::bulk_wait_read();
+            if (tid == 0) {  // complete before the count that publishes it (after the item)
+              umma::bulk_s2g(w.part + ((int64_t)b * A + piece) * G * PR, tile_a, kPartBytes);
+              umma::bulk_wait_done();
             }
+            pending = w.att_cnt + b;
           } else {
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              const float inv = scale_of(h);
-#pragma unroll
-              for (int bi = 0; bi < 2; ++bi) dst[h * DV + dim_of(bi)] = __float2bfloat16(o[bi][h] * inv);
-            }
-          }
-        };
-        if (Ab == 1) {
-          store_out([&](int h) { return s_ml[4 * h + 1] > 0.0f ? 1.0f / s_ml[4 * h + 1] : 0.0f; });
-          if (spart == 0 && p.lse)
-            p.lse[orow + sh] = Le_run > 0.0f ? (M_run + log2f(Le_run)) * kLn2 : -INFINITY;
-          if (tid == 0 && nch > 0) w.unit_done[b] = 0;
-        } else if (piece < Ab - 1) {
-          // publish this piece's partial and move on: the request's last piece merges them
-#pragma unroll
-          for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int bi = 0; bi < 2; ++bi) tile[h * PR + dim_of(bi)] = o[bi][h];
-          if (spart == 0) {
-            tile[sh * PR + DV] = M_run;
-            tile[sh * PR + DV + 1] = L_run;
-            tile[sh * PR + DV + 2] = Le_run;
-            tile[sh * PR + DV + 3] = 0.0f;
-          }
-          umma::fence_async_smem();
-          __syncthreads();
-          if (tid == 0) {  // complete before the count that publishes it (after the item)
-            umma::bulk_s2g(w.part + ((int64_t)b * A + piece) * G * PR, tile_a, kPartBytes);
-            umma::bulk_wait_done();
-          }
-          pending = w.att_cnt + b;
-        } else {
-          // the last piece: wait for the other Ab - 1 partials (claimed before this item, and
-          // they never wait on a later one), then fold them in one at a time: each lands in
-          // shared memory with one bulk copy, and the running maximum and sum move with it
-          if (tid == 0) s_misc[1] = mp_wait_at_least(w.att_cnt + b, Ab - 1, p.status) ? 1 : 0;
-          // per head: [0] maximum, [1] [2] the two sums, [3] [4] the factors of this step, [5] 1/L
-          float* s_mm = reinterpret_cast<float*>(region + Ls.mm);  // [G][8]
-          for (int g = tid; g < G; g += NT) {
-            s_mm[8 * g] = s_ml[4 * g];
-            s_mm[8 * g + 1] = s_ml[4 * g + 1];
-            s_mm[8 * g + 2] = s_ml[4 * g + 2];
-          }
-          __syncthreads();
-          if (s_misc[1]) {
-            const float* src = w.part + (int64_t)b * A * G * PR;
-            for (int q = 0; q < Ab - 1; ++q) {
-              if (tid == 0) {
-                umma::fence_async_global();
-                umma::mbar_expect_tx(bars_a + 24, kPartBytes);
-                umma::bulk_g2s(tile_a, src + (int64_t)q * G * PR, kPartBytes, bars_a + 24);
-              }
-              bar_wait(3);
-              for (int g = tid; g < G; g += NT) {
-                const float mq = tile[g * PR + DV];
-                const float M = s_mm[8 * g], Mn = fmaxf(M, mq);
-                const float fo = M == -INFINITY ? 0.0f : exp2f(M - Mn);
-                const float fq = mq == -INFINITY ? 0.0f : exp2f(mq - Mn);
-                s_mm[8 * g] = Mn;
-                s_mm[8 * g + 1] = fmaf(s_mm[8 * g + 1], fo, tile[g * PR + DV + 1] * fq);
-                s_mm[8 * g + 2] = fmaf(s_mm[8 * g + 2], fo, tile[g * PR + DV + 2] * fq);
-                s_mm[8 * g + 3] = fo;
-                s_mm[8 * g + 4] = fq;
-              }
-              __syncthreads();
-#pragma unroll
-              for (int h = 0; h < G; ++h) {
-                const float fo = s_mm[8 * h + 3], fq = s_mm[8 * h + 4];
-#pragma unroll
-                for (int bi = 0; bi < 2; ++bi)
-                  o[bi][h] = fmaf(tile[h * PR + dim_of(bi)], fq, o[bi][h] * fo);
-              }
-              __syncthreads();  // the tile is free for the next partial (or the output)
-            }
+            // the last piece: wait for the other Ab - 1 partials (claimed before this item, and
+            // they never wait on a later one), then fold them in one at a time: each lands in
+            // shared memory with one bulk copy, and the running maximum and sum move with it
+            if (tid == 0) s_misc[1] = mp_wait_at_least(w.att_cnt + b, Ab - 1, p.status) ? 1 : 0;
+            // per head: [0] maximum, [1] [2] the two sums, [3] [4] the factors of this step, [5] 1/L
+            float* s_mm = reinterpret_cast<float*>(region + Ls.mm);  // [G][8]
             for (int g = tid; g < G; g += NT) {
-              const float M = s_mm[8 * g], Lsum = s_mm[8 * g + 1], Le = s_mm[8 * g + 2];
-              s_mm[8 * g + 5] = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
-              if (p.lse) p.lse[orow + g] = Le > 0.0f ? (M + log2f(Le)) * kLn2 : -INFINITY;
+              s_mm[8 * g] = s_ml[4 * g];
+              s_mm[8 * g + 1] = s_ml[4 * g + 1];
+              s_mm[8 * g + 2] = s_ml[4 * g + 2];
             }
             __syncthreads();
-            store_out([&](int h) { return s_mm[8 * h + 5]; });
-            if (tid == 0) {  // every piece is past its waits: reset the request's counters
-              w.att_cnt[b] = 0;
-              w.unit_done[b] = 0;
+            if (s_misc[1]) {
+              const float* src = w.part + (int64_t)b * A * G * PR;
+              for (int q = 0; q < Ab - 1; ++q) {
+                if (tid == 0) {
+                  umma::fence_async_global();
+                  umma::mbar_expect_tx(bars_a + 24, kPartBytes);
+                  umma::bulk_g2s(tile_a, src + (int64_t)q * G * PR, kPartBytes, bars_a + 24);
+                }
+                bar_wait(3);
+                for (int g = tid; g < G; g += NT) {
+                  const float mq = tile[g * PR + DV];
+                  const float M = s_mm[8 * g], Mn = fmaxf(M, mq);
+                  const float fo = M == -INFINITY ? 0.0f : exp2f(M - Mn);
+                  const float fq = mq == -INFINITY ? 0.0f : exp2f(mq - Mn);
+                  s_mm[8 * g] = Mn;
+                  s_mm[8 * g + 1] = fmaf(s_mm[8 * g + 1], fo, tile[g * PR + DV + 1] * fq);
+                  s_mm[8 * g + 2] = fmaf(s_mm[8 * g + 2], fo, tile[g * PR + DV + 2] * fq);
+                  s_mm[8 * g + 3] = fo;
+                  s_mm[8 * g + 4] = fq;
+                }
+                __syncthreads();
+  #pragma unroll
+                for (int h = 0; h < G; ++h) {
+                  const float fo = s_mm[8 * h + 3], fq = s_mm[8 * h + 4];
+  #pragma unroll
+                  for (int bi = 0; bi < 2; ++bi)
+                    o[bi][h] = fmaf(tile[h * PR + dim_of(bi)], fq, o[bi][h] * fo);
+                }
+                __syncthreads();  // the tile is free for the next partial (or the output)
+              }
+              for (int g = tid; g < G; g += NT) {
+                const float M = s_mm[8 * g], Lsum = s_mm[8 * g + 1], Le = s_mm[8 * g + 2];
+                s_mm[8 * g + 5] = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
+                if (p.lse) p.lse[orow + g] = Le > 0.0f ? (M + log2f(Le)) * kLn2 : -INFINITY;
+              }
+              __syncthreads();
+              store_out([&](int h) { return s_mm[8 * h + 5]; });
+              if (tid == 0) {  // every piece is past its waits: reset the request's counters
+                w.att_cnt[b] = 0;
+                w.unit_done[b] = 0;
+              }
             }
           }
         }
@@ -1041,10 +1067,10 @@ int mla_persist_smem_bytes(const DecodeParams& p, int G) {
 
 int mla_persist_max_batch() { return kMpMaxB; }
 
-template <int G>
+template <int G, int MODE>
 static cudaError_t launch_mla_persist_t(const DecodeParams& p, const MpWs& w, int sm_count,
                                         cudaStream_t stream) {
-  auto kern = persist_mla_kernel<G>;
+  auto kern = persist_mla_kernel<G, MODE>;
   const int smem = mp_smem_layout(G, p.B, w.g).total;
   static std::atomic<int> optin[64];
   cudaError_t e = ensure_smem_optin(kern, smem, false, optin);
@@ -1067,10 +1093,11 @@ static cudaError_t launch_mla_persist_t(const DecodeParams& p, const MpWs& w, in
   return cudaLaunchKernelEx(&cfg, kern, p, w);
 }
 
-// The fused MLA call on `ws` (mla_persist_workspace_bytes() bytes for the same unit_cap,
-// counters zero): as many CTAs as fit on the sm_count SMs at once.
+// The MLA call (fused, select-only or decode-only, by `mode`) on `ws`
+// (mla_persist_workspace_bytes() bytes for the same unit_cap, counters zero): as many CTAs as
+// fit on the sm_count SMs at once.
 cudaError_t launch_mla_persist(const DecodeParams& p, int G, void* ws, int64_t unit_cap,
-                               int sm_count, cudaStream_t s) {
+                               int sm_count, cudaStream_t s, int mode) {
   const MpWsLayout L = mp_ws_layout(p, G, unit_cap);
   unsigned char* base = static_cast<unsigned char*>(ws);
   MpWs w;
@@ -1082,8 +1109,15 @@ cudaError_t launch_mla_persist(const DecodeParams& p, int G, void* ws, int64_t u
   w.cpid = reinterpret_cast<int32_t*>(base + L.cpid);
   w.part = reinterpret_cast<float*>(base + L.part);
   w.g = mp_geom(p.pt_stride, p.topk, p.bos, p.eos, p.kmax);
-  if (G == 16) return launch_mla_persist_t<16>(p, w, sm_count, s);
-  if (G == 32) return launch_mla_persist_t<32>(p, w, sm_count, s);
+  if (mode != kFused && mode != kSelect && mode != kDecode) return cudaErrorInvalidValue;
+  if (G == 16)
+    return mode == kFused    ? launch_mla_persist_t<16, kFused>(p, w, sm_count, s)
+           : mode == kSelect ? launch_mla_persist_t<16, kSelect>(p, w, sm_count, s)
+                             : launch_mla_persist_t<16, kDecode>(p, w, sm_count, s);
+  if (G == 32)
+    return mode == kFused    ? launch_mla_persist_t<32, kFused>(p, w, sm_count, s)
+           : mode == kSelect ? launch_mla_persist_t<32, kSelect>(p, w, sm_count, s)
+                             : launch_mla_persist_t<32, kDecode>(p, w, sm_count, s);
   return cudaErrorInvalidValue;
 }
 

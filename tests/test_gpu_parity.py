@@ -287,6 +287,29 @@ def test_bad_inputs_set_status_and_spare_other_units(oracle):
     assert torch.all(out[2, :c.G].float() == 0)
 
 
+def test_mla_decode_workspace_rejects_bad_selection(oracle):
+    """The MLA decode-only persistent launch: a selection entry past its request's pages is
+    reported and zeroes that request's outputs; the other requests still match the oracle."""
+    w = _case("c4s")
+    c = w["config"]
+    _, ref = _reference("c4s")
+    d = to_device(w)
+    bad_sel = ref["sel"].clone().cuda()
+    bad_sel[1, 0, 3] = 10 ** 6
+    ws = vt.decode_workspace(d["q"], d["k_pool"], d["v_pool"], d["page_table"], d["seq_lens"],
+                             bad_sel, head_dim_v=c.Dv)
+    assert ws is not None
+    st = _status()
+    out, lse = vt.vt_sparse_decode(d["q"], d["k_pool"], d["v_pool"], d["page_table"],
+                                   d["seq_lens"], bad_sel, ref["n_sel"].cuda(), c.sm_scale,
+                                   status=st, head_dim_v=c.Dv, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(st.item()) == vt.VT_DEV_BAD_SEL
+    assert torch.all(out[1].float() == 0)
+    keep = [0, 2]
+    compare_outputs(out[keep], lse[keep], ref["out"][keep], ref["lse"][keep])
+
+
 @pytest.mark.parametrize("name", ["c2s", "c4s", "c5s"])
 def test_last_page_centroid_is_never_read(name):
     """With eos >= 1 a request's last page is reserved, so no score reads its centroid: the
@@ -322,8 +345,8 @@ def test_last_page_centroid_is_never_read(name):
 
 @pytest.mark.parametrize("name", list(CASES))
 def test_select_and_decode_with_workspace(name, oracle):
-    """vt_select_pages_ws and vt_sparse_decode_ws (the persistent kernel's select-only and
-    decode-only launches for GQA heads, B <= 2048; the other shapes keep the cluster kernels)
+    """vt_select_pages_ws and vt_sparse_decode_ws (the persistent kernels' select-only and
+    decode-only launches, GQA and MLA, B <= 2048; larger batches keep the cluster kernels)
     against the oracle, twice in a row on the same workspaces."""
     w = _case(name)
     c = w["config"]
