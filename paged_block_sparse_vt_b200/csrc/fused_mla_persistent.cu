@@ -28,6 +28,9 @@
 //                   landing while the other round computes.  With several pieces, the earlier
 //                   ones take whole rounds and publish fp32 partials with one bulk copy each;
 //                   the last piece folds them in and writes the request's rows.
+// The same kernel, instantiated per mode, serves the select-only call (scan items, then one
+// merge item per request that writes its selection) and the decode-only call (attention items
+// only, each reading and checking its request's selection).
 // Queue, claims and counters work as in the GQA persistent kernel (fused_persistent.cu).
 #include "centroid_chunk.cuh"
 #include "decode_params.cuh"
